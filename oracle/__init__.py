@@ -1,0 +1,152 @@
+"""Float64 CPU oracle for exact attention (ctypes wrapper over attn_oracle.cpp).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the bench's CPU
+baseline leg may import this package; the product library never does. It
+shares no code with the CUDA path. Inputs are torch CPU tensors (bf16, f32 or
+f64); bf16 values are widened to double inside the C++ code.
+
+Parity pins (tests/test_oracle_pins.py) tie every function here to facts the
+pages and mathematics fix; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .build import build_oracle, library_path
+
+_lib = None
+_DT = {torch.float64: 0, torch.bfloat16: 1, torch.float32: 2}
+
+
+def _load(plant: int = 0):
+    global _lib
+    if plant:
+        return _bind(ctypes.CDLL(build_oracle(plant=plant)))
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            build_oracle()
+        _lib = _bind(ctypes.CDLL(path))
+    return _lib
+
+
+def _bind(lib):
+    P, I, D, L = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_int64
+    lib.oracle_attention_rows.argtypes = [I, P, P, P, I, I, I, I, I, I, I, D, P, L, P, P, P, I]
+    lib.oracle_attention_rows.restype = I
+    lib.oracle_attention_blockwise_rows.argtypes = [I, P, P, P, I, I, I, I, I, I, I, D, I, P, L, P, P, I]
+    lib.oracle_attention_blockwise_rows.restype = I
+    lib.oracle_decode_partials.argtypes = [I, P, P, P, I, I, I, I, I, I, I, D, P, P, I]
+    lib.oracle_decode_partials.restype = I
+    lib.oracle_combine.argtypes = [P, P, I, I, I, I, P, P]
+    lib.oracle_combine.restype = I
+    lib.oracle_hardware_threads.restype = I
+    return lib
+
+
+def _ptr(t: torch.Tensor):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ValueError(f"oracle {what}: invalid arguments (code {rc})")
+
+
+def hardware_threads() -> int:
+    return _load().oracle_hardware_threads()
+
+
+def _prep(q, k, v):
+    assert q.dtype == k.dtype == v.dtype and q.dtype in _DT
+    return q.contiguous(), k.contiguous(), v.contiguous(), _DT[q.dtype]
+
+
+def attention(q, k, v, causal: bool, scale: float, rows=None, nthreads: int = 0,
+              want_probs: bool = False, plant: int = 0):
+    """Direct definition. q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d].
+
+    Returns (o, lse[, probs]) as float64. With ``rows`` (flat indices
+    (b*Hq+h)*Nq+i) only those rows are computed: o [R,d], lse [R].
+    """
+    q, k, v, dt = _prep(q, k, v)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    full = rows is None
+    if full:
+        rows = torch.arange(B * Hq * Nq, dtype=torch.int64)
+    rows = rows.to(torch.int64).contiguous()
+    R = rows.numel()
+    o = torch.empty(R, d, dtype=torch.float64)
+    lse = torch.empty(R, dtype=torch.float64)
+    probs = torch.empty(R, Nk, dtype=torch.float64) if want_probs else None
+    rc = _load(plant).oracle_attention_rows(dt, _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Nq, Nk, d,
+                                            int(causal), float(scale), _ptr(rows), R, _ptr(o),
+                                            _ptr(lse), _ptr(probs) if want_probs else None, nthreads)
+    _check(rc, "attention")
+    if full:
+        o, lse = o.view(B, Hq, Nq, d), lse.view(B, Hq, Nq)
+        if want_probs:
+            probs = probs.view(B, Hq, Nq, Nk)
+    return (o, lse, probs) if want_probs else (o, lse)
+
+
+def attention_blockwise(q, k, v, causal: bool, scale: float, block_k: int, rows=None,
+                        nthreads: int = 0, plant: int = 0):
+    """The tiled online-softmax recurrence; same shapes and returns as attention()."""
+    q, k, v, dt = _prep(q, k, v)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    full = rows is None
+    if full:
+        rows = torch.arange(B * Hq * Nq, dtype=torch.int64)
+    rows = rows.to(torch.int64).contiguous()
+    R = rows.numel()
+    o = torch.empty(R, d, dtype=torch.float64)
+    lse = torch.empty(R, dtype=torch.float64)
+    rc = _load(plant).oracle_attention_blockwise_rows(dt, _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Nq,
+                                                      Nk, d, int(causal), float(scale), int(block_k),
+                                                      _ptr(rows), R, _ptr(o), _ptr(lse), nthreads)
+    _check(rc, "attention_blockwise")
+    if full:
+        return o.view(B, Hq, Nq, d), lse.view(B, Hq, Nq)
+    return o, lse
+
+
+def decode_partials(q, k, v, scale: float, num_splits: int, chunk: int, nthreads: int = 0,
+                    plant: int = 0):
+    """q [B,Hq,d], k/v [B,Hkv,L,d] -> o_part [B,Hq,S,d], lse_part [B,Hq,S] (float64)."""
+    q, k, v, dt = _prep(q, k, v)
+    B, Hq, d = q.shape
+    Hkv, L = k.shape[1], k.shape[2]
+    o = torch.empty(B, Hq, num_splits, d, dtype=torch.float64)
+    lse = torch.empty(B, Hq, num_splits, dtype=torch.float64)
+    rc = _load(plant).oracle_decode_partials(dt, _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, L, d,
+                                             num_splits, chunk, float(scale), _ptr(o), _ptr(lse),
+                                             nthreads)
+    _check(rc, "decode_partials")
+    return o, lse
+
+
+def combine(o_part, lse_part, plant: int = 0):
+    """o_part [B,Hq,S,d], lse_part [B,Hq,S] -> o [B,Hq,d], lse [B,Hq] (float64)."""
+    o_part = o_part.to(torch.float64).contiguous()
+    lse_part = lse_part.to(torch.float64).contiguous()
+    B, Hq, S, d = o_part.shape
+    o = torch.empty(B, Hq, d, dtype=torch.float64)
+    lse = torch.empty(B, Hq, dtype=torch.float64)
+    rc = _load(plant).oracle_combine(_ptr(o_part), _ptr(lse_part), B, Hq, S, d, _ptr(o), _ptr(lse))
+    _check(rc, "combine")
+    return o, lse
+
+
+def decode(q, k, v, scale: float, rows=None, nthreads: int = 0):
+    """Single-query decode by the direct definition: q [B,Hq,d] sees all L keys."""
+    B, Hq, d = q.shape
+    o, lse = attention(q.unsqueeze(2), k, v, False, scale, rows=rows, nthreads=nthreads)
+    if rows is None:
+        return o.view(B, Hq, d), lse.view(B, Hq)
+    return o, lse

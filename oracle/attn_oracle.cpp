@@ -1,0 +1,286 @@
+// Float64 CPU oracle for exact scaled-dot-product attention.
+//
+// TEST INFRASTRUCTURE ONLY. Nothing on the product path may link, load or call
+// this file: only the tests, the smoke check and the bench's CPU-baseline leg
+// use it. It shares no code, header or constant with the CUDA library.
+//
+// What it computes follows "1-Flash-Attention.md" (huajishe.fun), section
+// "问题分析" (standard attention: S = Q K^T, A = softmax(S / sqrt(d)), O = A V on
+// (batch, heads, seq_len, head_dim) tensors), with the caller's softmax scale in
+// place of 1/sqrt(d) (section "框架集成", softmax_scale). Every value is widened
+// to double before any arithmetic and nothing is rounded on the way out.
+//
+// Readings where the pages are silent (each also listed in the design notes):
+//  * causal: query row i sees key j iff j <= i (prefill has Nq == Nk);
+//  * LSE_i = ln sum_{j visible} exp(scale * q_i . k_j)  (natural log, scale in);
+//  * GQA/MQA: query head h reads key/value head h / (Hq / Hkv) (consecutive
+//    query heads share one key/value head);
+//  * split-KV partials are normalised: O_s = sum_s p v / l_s with lse_s; an
+//    empty split has lse_s = -inf, O_s = 0 and weight 0 in the merge.
+//
+// Functions:
+//  oracle_attention_rows            direct definition, selected rows
+//  oracle_attention_blockwise_rows  the tiled online-softmax recurrence
+//                                   ("递归计算softmax" section) - must equal
+//                                   the direct definition
+//  oracle_decode_partials           per-split partial (O_s, lse_s)
+//  oracle_combine                   logsumexp-weighted merge of partials
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <thread>
+#include <vector>
+
+// ORACLE_PLANT selects one deliberate mistake for the mutation tests, which
+// check that the pins catch it; 0 (the default build) plants nothing.
+#ifndef ORACLE_PLANT
+#define ORACLE_PLANT 0
+#endif
+
+namespace {
+
+constexpr int kPlant = ORACLE_PLANT;
+
+enum InType { IN_F64 = 0, IN_BF16 = 1, IN_F32 = 2 };
+
+// bf16 -> double: a bf16 value is the top 16 bits of an IEEE float32.
+inline double load_elem(int dtype, const void* base, int64_t idx) {
+    switch (dtype) {
+        case IN_F64: return static_cast<const double*>(base)[idx];
+        case IN_F32: return static_cast<const float*>(base)[idx];
+        default: {
+            uint32_t bits = static_cast<uint32_t>(static_cast<const uint16_t*>(base)[idx]) << 16;
+            float f;
+            std::memcpy(&f, &bits, sizeof f);
+            return f;
+        }
+    }
+}
+
+struct Problem {
+    int dtype;
+    const void *q, *k, *v;
+    int B, Hq, Hkv, Nq, Nk, d, causal;
+    double scale;
+};
+
+// Visible keys of query row i: [0, Nk) or [0, i] when causal.
+inline int64_t visible_keys(const Problem& p, int64_t i) {
+    if (kPlant == 3) return p.causal ? std::min<int64_t>(i + 2, p.Nk) : p.Nk;  // off by one
+    if (kPlant == 8) return p.causal ? std::max<int64_t>(i, 1) : std::max(p.Nk - 1, 1);  // drops a key
+    return p.causal ? std::min<int64_t>(i + 1, p.Nk) : p.Nk;
+}
+
+// Query head h reads key/value head h / G.
+inline int64_t kv_head(const Problem& p, int64_t h) {
+    if (kPlant == 2) return h % p.Hkv;  // wrong GQA grouping
+    return h / (p.Hq / p.Hkv);
+}
+
+// s_j = scale * sum_t q[t] k_j[t] for the visible keys of one row.
+void scores(const Problem& p, int64_t b, int64_t h, int64_t i, std::vector<double>& s) {
+    const int64_t hk = kv_head(p, h);
+    const int64_t qoff = ((b * p.Hq + h) * p.Nq + i) * p.d;
+    const int64_t koff = (b * p.Hkv + hk) * static_cast<int64_t>(p.Nk) * p.d;
+    const int64_t J = visible_keys(p, i);
+    s.assign(J, 0.0);
+    for (int64_t j = 0; j < J; ++j) {
+        double acc = 0.0;
+        for (int t = 0; t < p.d; ++t) {
+            const int64_t kidx = (kPlant == 7) ? koff + t * p.Nk + j : koff + j * p.d + t;  // 7: K^T
+            acc += load_elem(p.dtype, p.q, qoff + t) * load_elem(p.dtype, p.k, kidx);
+        }
+        s[j] = (kPlant == 1) ? acc : p.scale * acc;  // 1: scale dropped
+    }
+}
+
+// Direct definition for one row: softmax over the visible scores, then A V.
+void direct_row(const Problem& p, int64_t row, double* o, double* lse, double* prob) {
+    const int64_t i = row % p.Nq;
+    const int64_t bh = row / p.Nq;
+    const int64_t h = bh % p.Hq, b = bh / p.Hq;
+    const int64_t hk = kv_head(p, h);
+    const int64_t voff = (b * p.Hkv + hk) * static_cast<int64_t>(p.Nk) * p.d;
+    std::vector<double> s;
+    scores(p, b, h, i, s);
+    const int64_t J = static_cast<int64_t>(s.size());
+    double m = -std::numeric_limits<double>::infinity();
+    for (double x : s) m = std::max(m, x);
+    double l = 0.0;
+    for (int64_t j = 0; j < J; ++j) { s[j] = std::exp(s[j] - m); l += s[j]; }
+    for (int t = 0; t < p.d; ++t) o[t] = 0.0;
+    for (int64_t j = 0; j < J; ++j) {
+        const double a = s[j] / l;
+        if (prob) prob[j] = a;
+        for (int t = 0; t < p.d; ++t) o[t] += a * load_elem(p.dtype, p.v, voff + j * p.d + t);
+    }
+    if (prob) for (int64_t j = J; j < p.Nk; ++j) prob[j] = 0.0;
+    *lse = (kPlant == 4) ? m + std::log2(l) : m + std::log(l);  // 4: log base 2
+}
+
+// The page's block recurrence, keys visited in blocks of Bk:
+//   rowmax = max_j S_ij;  P_ij = exp(S_ij - rowmax)
+//   m_new = max(m_old, rowmax)
+//   d_new = d_old * exp(m_old - m_new) + exp(rowmax - m_new) * sum_j P_ij
+//   O_new = O_old * exp(m_old - m_new) + exp(rowmax - m_new) * (P_ij @ V_j)
+// and the normalisation O / d once at the end.
+void blockwise_row(const Problem& p, int64_t row, int Bk, double* o, double* lse) {
+    const int64_t i = row % p.Nq;
+    const int64_t bh = row / p.Nq;
+    const int64_t h = bh % p.Hq, b = bh / p.Hq;
+    const int64_t hk = kv_head(p, h);
+    const int64_t voff = (b * p.Hkv + hk) * static_cast<int64_t>(p.Nk) * p.d;
+    std::vector<double> s;
+    scores(p, b, h, i, s);
+    const int64_t J = static_cast<int64_t>(s.size());
+    double m_old = -std::numeric_limits<double>::infinity();
+    double d_old = 0.0;
+    std::vector<double> acc(p.d, 0.0), pv(p.d);
+    for (int64_t j0 = 0; j0 < J; j0 += Bk) {
+        const int64_t j1 = std::min<int64_t>(J, j0 + Bk);
+        double rowmax = -std::numeric_limits<double>::infinity();
+        for (int64_t j = j0; j < j1; ++j) rowmax = std::max(rowmax, s[j]);
+        double psum = 0.0;
+        std::fill(pv.begin(), pv.end(), 0.0);
+        for (int64_t j = j0; j < j1; ++j) {
+            const double pij = std::exp(s[j] - rowmax);
+            psum += pij;
+            for (int t = 0; t < p.d; ++t) pv[t] += pij * load_elem(p.dtype, p.v, voff + j * p.d + t);
+        }
+        const double m_new = std::max(m_old, rowmax);
+        double f_old = (d_old == 0.0) ? 0.0 : std::exp(m_old - m_new);
+        if (kPlant == 5 && d_old != 0.0) f_old = 1.0;  // 5: old state not rescaled
+        const double f_blk = std::exp(rowmax - m_new);
+        const double d_new = d_old * f_old + f_blk * psum;
+        for (int t = 0; t < p.d; ++t) acc[t] = acc[t] * f_old + f_blk * pv[t];
+        m_old = m_new;
+        d_old = d_new;
+    }
+    for (int t = 0; t < p.d; ++t) o[t] = acc[t] / d_old;
+    *lse = m_old + std::log(d_old);
+}
+
+int resolve_threads(int nthreads) {
+    if (nthreads > 0) return nthreads;
+    unsigned hc = std::thread::hardware_concurrency();
+    return hc ? static_cast<int>(hc) : 1;
+}
+
+template <class F>
+void parallel_rows(int64_t nrows, int nthreads, F fn) {
+    nthreads = static_cast<int>(std::min<int64_t>(resolve_threads(nthreads), std::max<int64_t>(nrows, 1)));
+    if (nthreads <= 1) { for (int64_t r = 0; r < nrows; ++r) fn(r); return; }
+    std::vector<std::thread> pool;
+    for (int t = 0; t < nthreads; ++t)
+        pool.emplace_back([=] { for (int64_t r = t; r < nrows; r += nthreads) fn(r); });
+    for (auto& th : pool) th.join();
+}
+
+int check(const Problem& p) {
+    if (p.B < 1 || p.Hq < 1 || p.Hkv < 1 || p.Nq < 1 || p.Nk < 1 || p.d < 1) return 1;
+    if (p.Hq % p.Hkv != 0) return 2;
+    if (p.causal && p.Nq != p.Nk) return 3;
+    return 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+int oracle_hardware_threads() { return resolve_threads(0); }
+
+// Direct attention for `nrows` rows; rows[r] = (b*Hq + h)*Nq + i.
+// o: nrows x d, lse: nrows, prob (optional): nrows x Nk. Returns 0 on success.
+int oracle_attention_rows(int dtype, const void* q, const void* k, const void* v,
+                          int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, double scale,
+                          const int64_t* rows, int64_t nrows, double* o, double* lse, double* prob,
+                          int nthreads) {
+    Problem p{dtype, q, k, v, B, Hq, Hkv, Nq, Nk, d, causal, scale};
+    if (int e = check(p)) return e;
+    const int64_t total = static_cast<int64_t>(B) * Hq * Nq;
+    for (int64_t r = 0; r < nrows; ++r) if (rows[r] < 0 || rows[r] >= total) return 4;
+    parallel_rows(nrows, nthreads, [&](int64_t r) {
+        direct_row(p, rows[r], o + r * d, lse + r, prob ? prob + r * static_cast<int64_t>(Nk) : nullptr);
+    });
+    return 0;
+}
+
+// The blockwise online-softmax recurrence with key block size block_k.
+int oracle_attention_blockwise_rows(int dtype, const void* q, const void* k, const void* v,
+                                    int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                                    double scale, int block_k, const int64_t* rows, int64_t nrows,
+                                    double* o, double* lse, int nthreads) {
+    Problem p{dtype, q, k, v, B, Hq, Hkv, Nq, Nk, d, causal, scale};
+    if (int e = check(p)) return e;
+    if (block_k < 1) return 5;
+    const int64_t total = static_cast<int64_t>(B) * Hq * Nq;
+    for (int64_t r = 0; r < nrows; ++r) if (rows[r] < 0 || rows[r] >= total) return 4;
+    parallel_rows(nrows, nthreads, [&](int64_t r) { blockwise_row(p, rows[r], block_k, o + r * d, lse + r); });
+    return 0;
+}
+
+// Split-KV partials for single-query decode: q [B,Hq,d], k/v [B,Hkv,L,d].
+// Split s covers keys [s*chunk, min(L, (s+1)*chunk)).
+// o_part [B,Hq,S,d] (normalised), lse_part [B,Hq,S]; empty split -> 0 / -inf.
+int oracle_decode_partials(int dtype, const void* q, const void* k, const void* v,
+                           int B, int Hq, int Hkv, int L, int d, int num_splits, int chunk,
+                           double scale, double* o_part, double* lse_part, int nthreads) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || d < 1 || num_splits < 1 || chunk < 1) return 1;
+    if (Hq % Hkv != 0) return 2;
+    const int64_t G = Hq / Hkv;
+    const int64_t units = static_cast<int64_t>(B) * Hq * num_splits;
+    parallel_rows(units, nthreads, [&](int64_t u) {
+        const int64_t s = u % num_splits, bh = u / num_splits;
+        const int64_t h = bh % Hq, b = bh / Hq, hk = h / G;
+        const int64_t j0 = s * chunk, j1 = std::min<int64_t>(L, j0 + chunk);
+        double* o = o_part + u * d;
+        for (int t = 0; t < d; ++t) o[t] = 0.0;
+        if (j0 >= j1) { lse_part[u] = -std::numeric_limits<double>::infinity(); return; }
+        const int64_t qoff = bh * d;
+        const int64_t kvoff = (b * Hkv + hk) * static_cast<int64_t>(L) * d;
+        std::vector<double> sc(j1 - j0);
+        double m = -std::numeric_limits<double>::infinity();
+        for (int64_t j = j0; j < j1; ++j) {
+            double acc = 0.0;
+            for (int t = 0; t < d; ++t)
+                acc += load_elem(dtype, q, qoff + t) * load_elem(dtype, k, kvoff + j * d + t);
+            sc[j - j0] = scale * acc;
+            m = std::max(m, sc[j - j0]);
+        }
+        double l = 0.0;
+        for (auto& x : sc) { x = std::exp(x - m); l += x; }
+        for (int64_t j = j0; j < j1; ++j)
+            for (int t = 0; t < d; ++t)
+                o[t] += (kPlant == 9 ? sc[j - j0] : sc[j - j0] / l) * load_elem(dtype, v, kvoff + j * d + t);
+        lse_part[u] = m + std::log(l);
+    });
+    return 0;
+}
+
+// Logsumexp-weighted merge: M = max_s lse_s, w_s = exp(lse_s - M),
+// O = sum_s w_s O_s / sum_s w_s, LSE = M + ln sum_s w_s.
+int oracle_combine(const double* o_part, const double* lse_part, int B, int Hq, int num_splits,
+                   int d, double* o, double* lse) {
+    if (B < 1 || Hq < 1 || num_splits < 1 || d < 1) return 1;
+    for (int64_t bh = 0; bh < static_cast<int64_t>(B) * Hq; ++bh) {
+        const double* ls = lse_part + bh * num_splits;
+        double M = -std::numeric_limits<double>::infinity();
+        for (int s = 0; s < num_splits; ++s) M = std::max(M, ls[s]);
+        double wsum = 0.0;
+        for (int t = 0; t < d; ++t) o[bh * d + t] = 0.0;
+        if (M == -std::numeric_limits<double>::infinity()) { lse[bh] = M; continue; }
+        for (int s = 0; s < num_splits; ++s) {
+            if (ls[s] == -std::numeric_limits<double>::infinity()) continue;
+            const double w = (kPlant == 6) ? 1.0 : std::exp(ls[s] - M);  // 6: plain average
+            wsum += w;
+            for (int t = 0; t < d; ++t) o[bh * d + t] += w * o_part[(bh * num_splits + s) * d + t];
+        }
+        for (int t = 0; t < d; ++t) o[bh * d + t] /= wsum;
+        lse[bh] = M + std::log(wsum);
+    }
+    return 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,248 @@
+"""Pins for the float64 oracle: facts fixed by the pages and by mathematics.
+
+None of these re-types the oracle's own formula. Each pin compares the oracle
+with something independent of it: a closed form, an invariant of the
+definition, an independent library routine (torch's float64 CPU
+scaled_dot_product_attention, scipy's softmax / logsumexp), or another
+oracle function that follows a different algorithm (the blockwise online
+recurrence of the "递归计算softmax" section of "1-Flash-Attention.md").
+
+The mutation test at the bottom builds oracle variants with one planted
+mistake each (a dropped scale, a wrong GQA grouping, a causal off-by-one, a
+log2 LSE, a missing rescale, a plain-average merge, a transposed K, a dropped
+key, unnormalised partials) and checks that at least one pin fails on each.
+"""
+import math
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+import torch.nn.functional as F
+
+import oracle
+
+TOL = 1e-12
+
+
+def _rand(seed, *shape):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(*shape, generator=g, dtype=torch.float64)
+
+
+def _sdpa(q, k, v, causal, scale):
+    return F.scaled_dot_product_attention(q, k, v, is_causal=causal, scale=scale, enable_gqa=True)
+
+
+def _lse_lib(q, k, causal, scale):
+    """LSE by scipy's logsumexp over masked scores (library routine)."""
+    B, Hq, N, d = q.shape
+    G = Hq // k.shape[1]
+    kk = k.repeat_interleave(G, dim=1)
+    s = (q @ kk.transpose(-1, -2)).numpy() * scale
+    if causal:
+        mask = np.triu(np.ones((N, k.shape[2]), dtype=bool), 1)
+        s = np.where(mask, -np.inf, s)
+    return torch.from_numpy(scipy.special.logsumexp(s, axis=-1))
+
+
+# ---------------------------------------------------------------- pins ----
+
+def pin_probs_are_distributions(plant=0):
+    """Softmax rows are probability vectors; causal rows put no mass past i."""
+    q, k, v = _rand(1, 1, 2, 9, 4), _rand(2, 1, 2, 9, 4), _rand(3, 1, 2, 9, 4)
+    for causal in (False, True):
+        _, _, p = oracle.attention(q, k, v, causal, 0.7, want_probs=True, plant=plant)
+        assert torch.all(p >= 0)
+        assert torch.allclose(p.sum(-1), torch.ones(1, 2, 9, dtype=torch.float64), atol=1e-14, rtol=0)
+        if causal:
+            assert torch.all(torch.triu(p[0, 0], 1) == 0)
+
+
+def pin_constant_v(plant=0):
+    """v_j = c for every j gives O_i = c for every row (weights sum to one)."""
+    q, k = _rand(4, 2, 3, 17, 8), _rand(5, 2, 3, 17, 8)
+    c = _rand(6, 8)
+    v = c.expand(2, 3, 17, 8).contiguous()
+    for causal in (False, True):
+        o, _ = oracle.attention(q, k, v, causal, 0.35, plant=plant)
+        assert torch.allclose(o, c.expand_as(o), atol=1e-14, rtol=0)
+
+
+def pin_causal_first_row(plant=0):
+    """Causal row 0 sees only key 0: O[0] = V[0], LSE[0] = scale * q0.k0."""
+    q, k, v = _rand(7, 1, 2, 12, 5), _rand(8, 1, 2, 12, 5), _rand(9, 1, 2, 12, 5)
+    o, lse = oracle.attention(q, k, v, True, 0.5, plant=plant)
+    assert torch.allclose(o[:, :, 0], v[:, :, 0], atol=1e-15, rtol=0)
+    dots = torch.tensor([[math.fsum((q[0, h, 0] * k[0, h, 0]).tolist()) for h in range(2)]], dtype=torch.float64)
+    assert torch.allclose(lse[:, :, 0], 0.5 * dots, atol=1e-14, rtol=0)
+
+
+def pin_single_key(plant=0):
+    """N = 1: the only key gets weight one, so O = V and LSE = scale * q.k."""
+    q, k, v = _rand(10, 3, 4, 1, 6), _rand(11, 3, 2, 1, 6), _rand(12, 3, 2, 1, 6)
+    for causal in (False, True):
+        o, lse = oracle.attention(q, k, v, causal, 1.3, plant=plant)
+        vv = v.repeat_interleave(2, dim=1)
+        kk = k.repeat_interleave(2, dim=1)
+        assert torch.allclose(o, vv, atol=1e-15, rtol=0)
+        assert torch.allclose(lse, 1.3 * (q * kk).sum(-1), atol=1e-13, rtol=0)
+
+
+def pin_two_keys_closed_form(plant=0):
+    """Scores {0, t*ln2}: weights 1/(1+2^t) and 2^t/(1+2^t), LSE = ln(1+2^t)."""
+    scale = 0.25
+    for t in (-3, 0, 1, 5):
+        q = torch.ones(1, 1, 2, 1, dtype=torch.float64)
+        k = torch.tensor([0.0, t * math.log(2) / scale], dtype=torch.float64).view(1, 1, 2, 1)
+        v = torch.tensor([2.0, -6.0], dtype=torch.float64).view(1, 1, 2, 1)
+        o, lse = oracle.attention(q, k, v, False, scale, plant=plant)
+        w1 = 2.0 ** t / (1 + 2.0 ** t)
+        want = (1 - w1) * 2.0 + w1 * -6.0
+        assert abs(o[0, 0, 0, 0].item() - want) < 1e-14
+        assert abs(lse[0, 0, 0].item() - math.log1p(2.0 ** t)) < 1e-14
+        # causal: row 0 sees key 0 only, row 1 sees both
+        o, lse = oracle.attention(q, k, v, True, scale, plant=plant)
+        assert abs(o[0, 0, 0, 0].item() - 2.0) < 1e-15
+        assert abs(o[0, 0, 1, 0].item() - want) < 1e-14
+
+
+def pin_identical_keys(plant=0):
+    """All keys equal: uniform weights, O = mean(V), LSE = s + ln(N)."""
+    N, d = 11, 3
+    q = _rand(13, 1, 1, N, d)
+    k = _rand(14, d).expand(1, 1, N, d).contiguous()
+    v = _rand(15, 1, 1, N, d)
+    o, lse = oracle.attention(q, k, v, False, 0.9, plant=plant)
+    assert torch.allclose(o[0, 0], v[0, 0].mean(0).expand(N, d), atol=1e-14, rtol=0)
+    s = 0.9 * (q[0, 0] @ k[0, 0, 0])
+    assert torch.allclose(lse[0, 0], s + math.log(N), atol=1e-13, rtol=0)
+
+
+def pin_library_sdpa(plant=0):
+    """Matches torch's float64 CPU SDPA (O) and scipy logsumexp (LSE), with GQA."""
+    cases = [(1, 1, 1, 7, 3), (2, 4, 2, 13, 5), (1, 6, 3, 9, 4), (1, 4, 1, 16, 8), (2, 2, 2, 5, 2)]
+    for i, (B, Hq, Hkv, N, d) in enumerate(cases):
+        q, k, v = _rand(20 + i, B, Hq, N, d), _rand(30 + i, B, Hkv, N, d), _rand(40 + i, B, Hkv, N, d)
+        for causal in (False, True):
+            scale = 0.3 + 0.2 * i
+            o, lse = oracle.attention(q, k, v, causal, scale, plant=plant)
+            assert torch.allclose(o, _sdpa(q, k, v, causal, scale), atol=1e-12, rtol=0)
+            assert torch.allclose(lse, _lse_lib(q, k, causal, scale), atol=1e-12, rtol=0)
+
+
+def pin_brute_force_tiny(plant=0):
+    """Exhaustive tiny shapes against scipy's softmax, row by row."""
+    seed = 100
+    for N in range(1, 6):
+        for d in (1, 2, 3):
+            for Hq, Hkv in ((1, 1), (2, 1), (2, 2), (4, 2)):
+                seed += 1
+                q, k, v = _rand(seed, 1, Hq, N, d), _rand(seed + 1000, 1, Hkv, N, d), _rand(seed + 2000, 1, Hkv, N, d)
+                for causal in (False, True):
+                    o, _ = oracle.attention(q, k, v, causal, 0.8, plant=plant)
+                    G = Hq // Hkv
+                    for h in range(Hq):
+                        for i in range(N):
+                            J = i + 1 if causal else N
+                            s = 0.8 * (k[0, h // G, :J] @ q[0, h, i]).numpy()
+                            want = scipy.special.softmax(s) @ v[0, h // G, :J].numpy()
+                            assert np.allclose(o[0, h, i].numpy(), want, atol=1e-13, rtol=0)
+
+
+def pin_blockwise_equals_direct(plant=0):
+    """The online recurrence over key blocks reaches the direct result for any block size."""
+    q, k, v = _rand(50, 2, 4, 70, 8), _rand(51, 2, 2, 70, 8), _rand(52, 2, 2, 70, 8)
+    q = q * 6  # large logits: the running max moves a lot between blocks
+    for causal in (False, True):
+        o, lse = oracle.attention(q, k, v, causal, 0.5, plant=plant)
+        for bk in (1, 3, 7, 64, 70):
+            ob, lb = oracle.attention_blockwise(q, k, v, causal, 0.5, bk, plant=plant)
+            assert torch.allclose(ob, o, atol=1e-12, rtol=1e-12)
+            assert torch.allclose(lb, lse, atol=1e-12, rtol=1e-12)
+
+
+def pin_invariants(plant=0):
+    """Joint key/value permutation, key shift and GQA replication invariants."""
+    B, Hq, Hkv, N, d = 1, 4, 2, 10, 6
+    q, k, v = _rand(60, B, Hq, N, d), _rand(61, B, Hkv, N, d), _rand(62, B, Hkv, N, d)
+    o, lse = oracle.attention(q, k, v, False, 0.6, plant=plant)
+    perm = torch.randperm(N, generator=torch.Generator().manual_seed(63))
+    op, lp = oracle.attention(q, k[:, :, perm].contiguous(), v[:, :, perm].contiguous(), False, 0.6, plant=plant)
+    assert torch.allclose(op, o, atol=1e-13, rtol=0) and torch.allclose(lp, lse, atol=1e-13, rtol=0)
+    u = _rand(64, d)
+    os_, ls_ = oracle.attention(q, (k + u).contiguous(), v, False, 0.6, plant=plant)
+    assert torch.allclose(os_, o, atol=1e-12, rtol=0)
+    assert torch.allclose(ls_, lse + 0.6 * (q @ u), atol=1e-12, rtol=0)
+    G = Hq // Hkv
+    for causal in (False, True):
+        og, lg = oracle.attention(q, k, v, causal, 0.6, plant=plant)
+        om, lm = oracle.attention(q, k.repeat_interleave(G, 1).contiguous(),
+                                  v.repeat_interleave(G, 1).contiguous(), causal, 0.6, plant=plant)
+        assert torch.equal(og, om) and torch.equal(lg, lm)
+        # shifting V of key/value head 1 by +1 moves exactly query heads G..2G-1 by +1
+        v2 = v.clone()
+        v2[:, 1] += 1.0
+        og2, _ = oracle.attention(q, k, v2, causal, 0.6, plant=plant)
+        assert torch.equal(og2[:, :G], og[:, :G])
+        assert torch.allclose(og2[:, G:], og[:, G:] + 1.0, atol=1e-13, rtol=0)
+
+
+def pin_decode_and_combine(plant=0):
+    """Decode = last row of causal prefill; merging any split of the keys = direct."""
+    B, Hq, Hkv, L, d = 2, 4, 2, 37, 5
+    q, k, v = _rand(70, B, Hq, L, d), _rand(71, B, Hkv, L, d), _rand(72, B, Hkv, L, d)
+    o_pre, l_pre = oracle.attention(q, k, v, True, 0.45, plant=plant)
+    qd = q[:, :, L - 1].contiguous()
+    od, ld = oracle.decode(qd, k, v, 0.45)
+    assert torch.allclose(od, o_pre[:, :, L - 1], atol=1e-13, rtol=0)
+    assert torch.allclose(ld, l_pre[:, :, L - 1], atol=1e-13, rtol=0)
+    for S, chunk in ((1, 37), (2, 19), (5, 8), (8, 5), (40, 1), (7, 8)):  # (7, 8): empty splits
+        op, lp = oracle.decode_partials(qd, k, v, 0.45, S, chunk, plant=plant)
+        oc, lc = oracle.combine(op, lp, plant=plant)
+        assert torch.allclose(oc, od, atol=1e-13, rtol=0)
+        assert torch.allclose(lc, ld, atol=1e-13, rtol=0)
+
+
+def pin_bf16_inputs_widen_exactly(plant=0):
+    """bf16 inputs give the same answer as the same values passed as float64."""
+    q, k, v = (_rand(s, 1, 2, 9, 8).to(torch.bfloat16) for s in (80, 81, 82))
+    ob, lb = oracle.attention(q, k, v, True, 0.3, plant=plant)
+    od, ld = oracle.attention(q.double(), k.double(), v.double(), True, 0.3, plant=plant)
+    assert torch.equal(ob, od) and torch.equal(lb, ld)
+
+
+def pin_row_sampling(plant=0):
+    """Computing a subset of rows gives exactly those rows of the full result."""
+    q, k, v = _rand(90, 2, 3, 20, 4), _rand(91, 2, 3, 20, 4), _rand(92, 2, 3, 20, 4)
+    o, lse = oracle.attention(q, k, v, True, 0.5, plant=plant)
+    rows = torch.tensor([0, 19, 20, 57, 119])
+    orr, lr = oracle.attention(q, k, v, True, 0.5, rows=rows, plant=plant)
+    assert torch.equal(orr, o.reshape(-1, 4)[rows]) and torch.equal(lr, lse.reshape(-1)[rows])
+
+
+PINS = [pin_probs_are_distributions, pin_constant_v, pin_causal_first_row, pin_single_key,
+        pin_two_keys_closed_form, pin_identical_keys, pin_library_sdpa, pin_brute_force_tiny,
+        pin_blockwise_equals_direct, pin_invariants, pin_decode_and_combine,
+        pin_bf16_inputs_widen_exactly, pin_row_sampling]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_pin(pin):
+    pin()
+
+
+PLANTS = {1: "scale dropped", 2: "GQA head h % Hkv", 3: "causal off by one", 4: "LSE in log2",
+          5: "recurrence without rescale", 6: "merge by plain average", 7: "K read transposed",
+          8: "one key dropped", 9: "partials not normalised"}
+
+
+@pytest.mark.parametrize("plant", sorted(PLANTS), ids=[PLANTS[p] for p in sorted(PLANTS)])
+def test_planted_mistake_is_caught(plant):
+    caught = []
+    for pin in PINS:
+        try:
+            pin(plant=plant)
+        except (AssertionError, ValueError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches planted mistake {plant} ({PLANTS[plant]})"
