@@ -1,0 +1,414 @@
+"""Benchmark of the exact-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole path over one batch of synthetic inputs:
+  1. attn_fwd, causal, on the LLaMA-7B-shaped prefill (B=2, H=32, N=2048, d=128)
+  2. attn_fwd, non-causal, same shape
+  3. attn_decode_splitkv + 4. attn_combine on single-query decode
+     (B=1, Hq=32, Hkv=8, L=131072, d=128; the default split count).
+The printed `value` is the causal prefill's TFLOPS (4*B*H*N^2*d/2 per launch
+over the kernel's CUDA-event time, summed over all ranks); the decode's KV-read
+GB/s is reported beside it. Inputs are seeded N(0,1) bf16, resident in HBM
+before the timed region. The 537 MB KV stream of the decode (and a 256 MB
+buffer write) run between consecutive prefill launches, so every launch starts
+with a cold L2 (126 MB).
+
+With N > 1 (launched under torch.distributed.run) every rank runs the same
+per-GPU workload on its own batch (weak scaling, no data-path collective); the
+elapsed time is the max over ranks.
+
+--impl reference times the float64 CPU oracle (the checker) on the host cores
+on a bounded sample of the same causal prefill workload; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import seeded_inputs as si  # noqa: E402
+
+METRIC = "attn fwd TFLOPS (% BF16 TC peak); split-KV decode GB/s (% HBM peak)"
+PREFILL = si.PrefillShape("llama7b B2 H32 N2048 d128", 2, 32, 32, 2048, 128, True, seed=1001)
+PREFILL_NC = si.PrefillShape("llama7b B2 H32 N2048 d128 non-causal", 2, 32, 32, 2048, 128, False, seed=1001)
+DECODE = si.DecodeShape("decode B1 Hq32 Hkv8 L131072 d128", 1, 32, 8, 131072, 128, seed=1004)
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch from one ncu capture, valid only for the kernel source
+# it was taken on (sha256 of the kernel file, first 16 hex digits).
+NCU_TRAFFIC = {}
+
+
+def kernel_sha(name: str) -> str:
+    path = os.path.join(ROOT, "exact_attention_ring_b200", "csrc", name)
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, flag in zip(names, parts[5:9]):
+                if flag.lower() in ("active", "1"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        loaded = [x for x in sm if x > 0.5 * (smax or max(sm))] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def physical_gpu(local: int) -> str:
+    """nvidia-smi's id (index or UUID) of this process's CUDA device."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local < len(ids):
+            return ids[local]
+    return str(local)
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+# ----------------------------------------------------------------- our arm --
+
+def run_ours(args):
+    import exact_attention_ring_b200 as eab
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    # inputs resident in HBM before timing (rank-specific seeds: independent batches)
+    p = PREFILL
+    q, k, v = (t.to(dev) for t in si.make_qkv(p.seed + 17 * rank, p.B, p.Hq, p.Hkv, p.N, p.d))
+    o = torch.empty_like(q)
+    lse = torch.empty(p.B, p.Hq, p.N, device=dev)
+    o2 = torch.empty_like(q)
+    lse2 = torch.empty_like(lse)
+    dc = DECODE
+    qd, kd, vd = (t.to(dev) for t in si.make_decode(dc.seed + 17 * rank, dc.B, dc.Hq, dc.Hkv, dc.L, dc.d))
+    S = eab.attn_decode_default_splits(dc.B, dc.Hq, dc.Hkv, dc.L)
+    o_part = torch.empty(dc.B, dc.Hq, S, dc.d, device=dev)
+    lse_part = torch.empty(dc.B, dc.Hq, S, device=dev)
+    od = torch.empty(dc.B, dc.Hq, dc.d, device=dev, dtype=torch.bfloat16)
+    lsed = torch.empty(dc.B, dc.Hq, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
+
+    n_ev = 5
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        eab.attn_fwd(q, k, v, o, lse, True, p.scale, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        eab.attn_fwd(q, k, v, o2, lse2, False, p.scale, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        eab.attn_decode_splitkv(qd, kd, vd, o_part, lse_part, S, dc.scale, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        eab.attn_combine(o_part, lse_part, od, lsed, stream)
+        if ev is not None:
+            ev[4].record(stream)
+        flush.fill_(float(rank))  # write > L2 so the next prefill starts cold
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert eab.attn_device_status() == 0
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(physical_gpu(local)) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(events[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = max_over_ranks(start.elapsed_time(end), world)
+    t_fwd_c = sum(e[0].elapsed_time(e[1]) for e in events) / args.steps
+    t_fwd_n = sum(e[1].elapsed_time(e[2]) for e in events) / args.steps
+    t_dec = sum(e[2].elapsed_time(e[3]) for e in events) / args.steps
+    t_comb = sum(e[3].elapsed_time(e[4]) for e in events) / args.steps
+    t_fwd_c, t_fwd_n, t_dec, t_comb = (max_over_ranks(x, world) for x in (t_fwd_c, t_fwd_n, t_dec, t_comb))
+    assert eab.attn_device_status() == 0
+
+    tflops_c = p.flops() / (t_fwd_c * 1e-3) / 1e12
+    tflops_n = PREFILL_NC.flops() / (t_fwd_n * 1e-3) / 1e12
+    kv_bytes = dc.kv_bytes()
+    dec_gbs = kv_bytes / ((t_dec + t_comb) * 1e-3) / 1e9
+    dec_kernel_gbs = kv_bytes / (t_dec * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers (causal prefill)
+    qh, kh, vh = (t.pin_memory() for t in si.make_qkv(p.seed + 17 * rank, p.B, p.Hq, p.Hkv, p.N, p.d))
+    oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    lh = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    def e2e_step():
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        eab.attn_fwd(q, k, v, o, lse, True, p.scale, stream)
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, 20))
+    barrier(world)
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(s2.elapsed_time(e2) / e2e_steps, world)
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+
+    # ---- roofline of each kernel; the dominant one goes in "roofline"
+    tc_peak = peaks["bf16_tflops"]
+    hbm_peak = peaks["hbm_gbs"]
+    fwd_sha = kernel_sha("attn_fwd_sm100.cuh")
+    dec_sha = kernel_sha("decode_sm100.cuh")
+    def traffic(name, sha):
+        rec = NCU_TRAFFIC.get(name)
+        return rec["bytes_per_launch"] if rec and rec["source_sha"] == sha else None
+    roof_fwd = {"kernel": "attn_fwd_kernel<128,causal>", "bound": "tensor", "achieved": round(tflops_c, 1),
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": round(tflops_c / tc_peak, 4),
+                "traffic": traffic("attn_fwd_causal", fwd_sha), "ms": round(t_fwd_c, 5),
+                "peak_source": f"{peak_src} bf16_tflops (burst)"}
+    roof_fwd_nc = {"kernel": "attn_fwd_kernel<128,noncausal>", "bound": "tensor", "achieved": round(tflops_n, 1),
+                   "peak": tc_peak, "unit": "TFLOP/s", "frac": round(tflops_n / tc_peak, 4),
+                   "traffic": traffic("attn_fwd_noncausal", fwd_sha), "ms": round(t_fwd_n, 5)}
+    roof_dec = {"kernel": "decode_splitkv_kernel<128,4>", "bound": "hbm", "achieved": round(dec_kernel_gbs, 1),
+                "peak": hbm_peak, "unit": "GB/s", "frac": round(dec_kernel_gbs / hbm_peak, 4),
+                "traffic": traffic("decode", dec_sha), "ms": round(t_dec, 5),
+                "peak_source": f"{peak_src} hbm_gbs"}
+    times = {"fwd_causal": t_fwd_c, "fwd_noncausal": t_fwd_n, "decode": t_dec}
+    dominant = max(times, key=times.get)
+    roofline = {"fwd_causal": roof_fwd, "fwd_noncausal": roof_fwd_nc, "decode": roof_dec}[dominant]
+
+    cpu = cpu_baseline_sample(budget_s=args.cpu_budget) if (rank == 0 and world == 1 and not args.no_cpu) else None
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": round(tflops_c * world, 2),
+            "unit": "TFLOPS",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1), bf16)",
+            "config": {
+                "workload": "prefill B2 H32 N2048 d128 causal (LLaMA-7B shape); step also runs the non-causal "
+                            "prefill and split-KV decode B1 Hq32 Hkv8 L131072 d128 + combine",
+                "prefill": {"B": p.B, "Hq": p.Hq, "Hkv": p.Hkv, "N": p.N, "d": p.d, "causal": True},
+                "decode": {"B": dc.B, "Hq": dc.Hq, "Hkv": dc.Hkv, "L": dc.L, "d": dc.d, "num_splits": S},
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                "l2": "inputs resident in HBM; a 256 MB buffer write and the 537 MB decode KV stream (> 126 MB L2) "
+                      "run between consecutive prefill launches",
+            },
+            "decode": {"value": round(dec_gbs * world, 1), "unit": "GB/s", "kernel_gbs": round(dec_kernel_gbs, 1),
+                       "frac_hbm": round(dec_kernel_gbs / hbm_peak, 4), "ms_decode": round(t_dec, 5),
+                       "ms_combine": round(t_comb, 5), "kv_bytes": kv_bytes},
+            "prefill_noncausal": {"value": round(tflops_n * world, 2), "unit": "TFLOPS",
+                                  "frac": round(tflops_n / tc_peak, 4)},
+            "roofline": roofline,
+            "kernels": {"fwd_causal": roof_fwd, "fwd_noncausal": roof_fwd_nc, "decode": roof_dec},
+            "e2e": {"value": round(p.flops() * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+            "peaks": {"source": peak_src, "bf16_tflops": tc_peak, "hbm_gbs": hbm_peak},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------ oracle timing --
+
+def _oracle_slices(n_slices, budget_s, seed_offset=0):
+    """Times the oracle on whole (b, h) slices of the causal prefill, stopping
+    after `budget_s` seconds or `n_slices` slices. Returns (flops, seconds, k)."""
+    import oracle
+    p = PREFILL
+    q, k, v = si.make_qkv(p.seed + seed_offset, p.B, p.Hq, p.Hkv, p.N, p.d)
+    per_slice = 4.0 * p.N * (p.N + 1) / 2 * p.d  # causal: row i sees i+1 keys
+    done, elapsed = 0, 0.0
+    order = torch.randperm(p.B * p.Hq, generator=torch.Generator().manual_seed(5)).tolist()
+    for s in order[:n_slices]:
+        rows = torch.arange(s * p.N, (s + 1) * p.N, dtype=torch.int64)
+        t0 = time.perf_counter()
+        oracle.attention(q, k, v, True, p.scale, rows=rows)
+        elapsed += time.perf_counter() - t0
+        done += 1
+        if elapsed >= budget_s:
+            break
+    return done * per_slice, elapsed, done
+
+
+def cpu_baseline_sample(budget_s=15.0):
+    import oracle
+    flops, secs, k = _oracle_slices(PREFILL.B * PREFILL.Hq, budget_s)
+    return {"value": flops / secs / 1e12, "unit": "TFLOPS", "cores": oracle.hardware_threads(), "kind": "oracle",
+            "sample": f"{k} of {PREFILL.B * PREFILL.Hq} (b,h) slices of the causal prefill B2 H32 N2048 d128, all "
+                      f"2048 rows each ({secs:.1f} s of float64 CPU work, all host threads)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    p = PREFILL
+    for _ in range(args.warmup):
+        _oracle_slices(1, 0.0)
+    flops, secs = 0.0, 0.0
+    for i in range(args.steps):
+        f, s, _ = _oracle_slices(1, 0.0, seed_offset=0)
+        flops += f
+        secs += s
+    val = flops / secs / 1e12
+    cores = oracle.hardware_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1), bf16 widened to f64)",
+        "config": {"workload": "prefill B2 H32 N2048 d128 causal (LLaMA-7B shape); one (b,h) slice per step",
+                   "prefill": {"B": p.B, "Hq": p.Hq, "Hkv": p.Hkv, "N": p.N, "d": p.d, "causal": True}},
+        "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                         "sample": "one (b,h) slice (2048 rows) of the causal prefill per step"},
+        "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,171 @@
+"""ctypes binding of the C ABI in include/attn.h (argument marshalling only)."""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "_lib", "libattn_b200.so")
+
+ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = range(5)
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {_status_name(status)}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"exact_attention_ring_b200: CUDA library not built ({_LIB_PATH}); "
+            "run `python -m exact_attention_ring_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.attn_fwd.restype = I
+    lib.attn_decode_splitkv.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.attn_decode_splitkv.restype = I
+    lib.attn_combine.argtypes = [P, P, P, P, I, I, I, I, P]
+    lib.attn_combine.restype = I
+    lib.attn_decode_default_splits.argtypes = [I, I, I, I]
+    lib.attn_decode_default_splits.restype = I
+    lib.attn_status_string.argtypes = [I]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    lib.attn_device_status.argtypes = [P]
+    lib.attn_device_status.restype = I
+    lib.attn_selftest_bounded_wait.argtypes = [I, P]
+    lib.attn_selftest_bounded_wait.restype = I
+    return lib
+
+
+_lib = _load()
+
+
+def _status_name(status: int) -> str:
+    return _lib.attn_status_string(int(status)).decode()
+
+
+def attn_status_string(status: int) -> str:
+    return _status_name(status)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(status: int, what: str):
+    if status != ATTN_OK:
+        raise AttnError(status, what)
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+# -------------------------------------------------------------- C ABI calls --
+
+def attn_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None):
+    """q [B,Hq,N,d], k/v [B,Hkv,N,d], o [B,Hq,N,d] bf16; lse [B,Hq,N] fp32."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, torch.bfloat16, n)
+    _need(lse, torch.float32, "lse")
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape or o.shape != q.shape or lse.shape != (B, Hq, N):
+        raise ValueError("attn_fwd: inconsistent shapes")
+    _check(_lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, int(bool(causal)),
+                         float(scale), _stream(stream)), "attn_fwd")
+
+
+def attn_decode_splitkv(q, k, v, o_part, lse_part, num_splits: int, scale: float, stream=None):
+    """q [B,Hq,d], k/v [B,Hkv,L,d] bf16; o_part [B,Hq,S,d], lse_part [B,Hq,S] fp32."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    _need(o_part, torch.float32, "o_part")
+    _need(lse_part, torch.float32, "lse_part")
+    B, Hq, d = q.shape
+    Hkv, L = k.shape[1], k.shape[2]
+    S = int(num_splits)
+    if k.shape != (B, Hkv, L, d) or v.shape != k.shape or o_part.shape != (B, Hq, S, d) \
+            or lse_part.shape != (B, Hq, S):
+        raise ValueError("attn_decode_splitkv: inconsistent shapes")
+    _check(_lib.attn_decode_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), B, Hq, Hkv, L, d,
+                                    S, float(scale), _stream(stream)), "attn_decode_splitkv")
+
+
+def attn_combine(o_part, lse_part, o, lse, stream=None):
+    """o_part [B,Hq,S,d], lse_part [B,Hq,S] fp32 -> o [B,Hq,d] bf16, lse [B,Hq] fp32."""
+    _need(o_part, torch.float32, "o_part")
+    _need(lse_part, torch.float32, "lse_part")
+    _need(o, torch.bfloat16, "o")
+    _need(lse, torch.float32, "lse")
+    B, Hq, S, d = o_part.shape
+    if lse_part.shape != (B, Hq, S) or o.shape != (B, Hq, d) or lse.shape != (B, Hq):
+        raise ValueError("attn_combine: inconsistent shapes")
+    _check(_lib.attn_combine(_ptr(o_part), _ptr(lse_part), _ptr(o), _ptr(lse), B, Hq, S, d, _stream(stream)),
+           "attn_combine")
+
+
+def attn_decode_default_splits(B: int, Hq: int, Hkv: int, L: int) -> int:
+    return int(_lib.attn_decode_default_splits(B, Hq, Hkv, L))
+
+
+def attn_device_status(stream=None) -> int:
+    """Synchronises the stream, returns (and clears) the device-side status."""
+    return int(_lib.attn_device_status(_stream(stream)))
+
+
+def attn_selftest_bounded_wait(limit_us: int, stream=None):
+    _check(_lib.attn_selftest_bounded_wait(int(limit_us), _stream(stream)), "attn_selftest_bounded_wait")
+
+
+def decode_chunk(L: int, num_splits: int) -> int:
+    """Keys per split used by attn_decode_splitkv: 32 * ceil(ceil(L / S) / 32)."""
+    per = -(-L // num_splits)
+    return -(-per // 32) * 32
+
+
+# ------------------------------------------------------------- convenience --
+
+def attention(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
+    """Allocates o, lse and runs attn_fwd. Returns (o bf16, lse fp32)."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)
+    attn_fwd(q, k, v, o, lse, causal, scale, stream)
+    return o, lse
+
+
+def decode(q, k, v, scale: float | None = None, num_splits: int | None = None, stream=None):
+    """Split-KV decode plus combine. q [B,Hq,d], k/v [B,Hkv,L,d] -> (o [B,Hq,d], lse [B,Hq])."""
+    B, Hq, d = q.shape
+    Hkv, L = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    S = num_splits or attn_decode_default_splits(B, Hq, Hkv, L)
+    o_part = torch.empty(B, Hq, S, d, device=q.device, dtype=torch.float32)
+    lse_part = torch.empty(B, Hq, S, device=q.device, dtype=torch.float32)
+    attn_decode_splitkv(q, k, v, o_part, lse_part, S, scale, stream)
+    o = torch.empty(B, Hq, d, device=q.device, dtype=torch.bfloat16)
+    lse = torch.empty(B, Hq, device=q.device, dtype=torch.float32)
+    attn_combine(o_part, lse_part, o, lse, stream)
+    return o, lse

@@ -1,0 +1,215 @@
+// C ABI of the exact-attention library (declared in include/attn.h).
+//
+// Every call checks its arguments on the host before anything is enqueued,
+// encodes the TMA tensor maps it needs (cuTensorMapEncodeTiled, fetched through
+// the runtime's driver entry point so the library does not link libcuda), and
+// launches on the caller's stream. The whole library is one translation unit so
+// that the kernels share a single device-side status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "attn_fwd_sm100.cuh"
+#include "decode_sm100.cuh"
+
+namespace eab {
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// bf16 tensor viewed as [planes, rows, D] with a {64, box_rows, 1} box and
+// 128-byte swizzle; rows past `rows` read as zero.
+bool make_map(CUtensorMap* map, const void* base, int D, int rows, int planes, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(rows), cuuint64_t(planes)};
+    const cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(D) * 2 * cuuint64_t(rows)};
+    const cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* ptr) { return ptr != nullptr && (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
+
+bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D, bool CAUSAL>
+attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                         cudaStream_t stream) {
+    using C = FwdCfg<D>;
+    auto kern = attn_fwd_kernel<D, CAUSAL>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    const long long grid = static_cast<long long>(p.n_qtiles) * p.B * p.Hq;
+    if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    kern<<<static_cast<unsigned>(grid), C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, int GH>
+attn_status_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                            cudaStream_t stream) {
+    using C = DecCfg<D, GH>;
+    auto kern = decode_splitkv_kernel<D, GH>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    const dim3 grid(p.S, p.Hkv * p.groups, p.B);
+    kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D>
+attn_status_t launch_decode_d(const CUtensorMap& tk, const CUtensorMap& tv, DecodeParams p, cudaStream_t stream) {
+    const int G = p.Hq / p.Hkv;
+    // heads per block: the largest of 4, 2, 1 that divides the group (the query
+    // heads live in registers; more than 4 heads of 128 columns would spill)
+    if (G % 4 == 0) { p.groups = G / 4; return launch_decode<D, 4>(tk, tv, p, stream); }
+    if (G % 2 == 0) { p.groups = G / 2; return launch_decode<D, 2>(tk, tv, p, stream); }
+    p.groups = G;
+    return launch_decode<D, 1>(tk, tv, p, stream);
+}
+
+// One thread waits on an mbarrier that nothing completes, with a short limit.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    mbar_wait(&bar, 0, &abort_flag, limit_ns);
+}
+
+}  // namespace
+}  // namespace eab
+
+using namespace eab;
+
+extern "C" {
+
+const char* attn_status_string(attn_status_t s) {
+    switch (s) {
+        case ATTN_OK: return "ATTN_OK";
+        case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+        case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+        case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+        case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    }
+    return "ATTN_ERR_UNKNOWN";
+}
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                       int N, int d, int causal, float scale, attn_stream_t stream) {
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return ATTN_ERR_INVALID_ARG;
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || (causal != 0 && causal != 1) || !scale_ok(scale))
+        return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (static_cast<long long>(B) * Hq > 65535LL * 1024) return ATTN_ERR_INVALID_ARG;
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, q, d, N, B * Hq, 128) || !make_map(&tk, k, d, N, B * Hkv, 128) ||
+        !make_map(&tv, v, d, N, B * Hkv, 128))
+        return ATTN_ERR_CUDA;
+    FwdParams p;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N;
+    p.n_qtiles = (N + 127) / 128;
+    p.scale_log2 = scale * kLog2e;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 128) return causal ? launch_fwd<128, true>(tq, tk, tv, p, st) : launch_fwd<128, false>(tq, tk, tv, p, st);
+    return causal ? launch_fwd<64, true>(tq, tk, tv, p, st) : launch_fwd<64, false>(tq, tk, tv, p, st);
+}
+
+attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
+                                  int B, int Hq, int Hkv, int L, int d, int num_splits, float scale,
+                                  attn_stream_t stream) {
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part) || !aligned16(lse_part))
+        return ATTN_ERR_INVALID_ARG;
+    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0 || num_splits < 1 || num_splits > L ||
+        !scale_ok(scale))
+        return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (B > 65535 || num_splits > 0x7fffffff / 2) return ATTN_ERR_INVALID_ARG;
+    const int per = (L + num_splits - 1) / num_splits;
+    const int chunk = (per + 31) / 32 * 32;
+    CUtensorMap tk, tv;
+    if (!make_map(&tk, k, d, L, B * Hkv, 32) || !make_map(&tv, v, d, L, B * Hkv, 32)) return ATTN_ERR_CUDA;
+    DecodeParams p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.o_part = o_part;
+    p.lse_part = lse_part;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.S = num_splits; p.chunk = chunk;
+    p.groups = 1;
+    p.scale_log2 = scale * kLog2e;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    return d == 128 ? launch_decode_d<128>(tk, tv, p, st) : launch_decode_d<64>(tk, tv, p, st);
+}
+
+attn_status_t attn_combine(const float* o_part, const float* lse_part, void* o, float* lse, int B, int Hq,
+                           int num_splits, int d, attn_stream_t stream) {
+    if (!aligned16(o_part) || !aligned16(lse_part) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_INVALID_ARG;
+    if (B < 1 || Hq < 1 || num_splits < 1) return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    const long long blocks = static_cast<long long>(B) * Hq;
+    const size_t smem = static_cast<size_t>(num_splits) * sizeof(float);
+    if (blocks > 0x7fffffffLL || smem > 48 * 1024) return ATTN_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
+    if (d == 128)
+        combine_kernel<128><<<static_cast<unsigned>(blocks), 128, smem, st>>>(o_part, lse_part, ob, lse, num_splits);
+    else
+        combine_kernel<64><<<static_cast<unsigned>(blocks), 64, smem, st>>>(o_part, lse_part, ob, lse, num_splits);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_decode_default_splits(int B, int Hq, int Hkv, int L) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0) return 0;
+    constexpr int kSMs = 148, kWaves = 2, kMinKeys = 256;
+    const int G = Hq / Hkv;
+    const int gh = (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
+    const long long units = static_cast<long long>(B) * Hkv * (G / gh);
+    long long s = (kSMs * kWaves + units - 1) / units;
+    const long long max_s = (L + kMinKeys - 1) / kMinKeys;
+    if (s > max_s) s = max_s;
+    if (s < 1) s = 1;
+    return static_cast<int>(s);
+}
+
+attn_status_t attn_device_status(attn_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+    int value = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&value, g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (value != 0 && cudaMemcpyToSymbol(g_attn_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    return value == 0 ? ATTN_OK : static_cast<attn_status_t>(value);
+}
+
+attn_status_t attn_selftest_bounded_wait(int limit_us, attn_stream_t stream) {
+    if (limit_us < 1 || limit_us > 1000000) return ATTN_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(uint64_t(limit_us) * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

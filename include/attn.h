@@ -1,0 +1,134 @@
+/*
+ * exact_attention_ring_b200 — C ABI of the B200 (sm_100a) exact-attention library.
+ *
+ * Exact scaled-dot-product attention O = softmax(scale * Q K^T) V, computed tile
+ * by tile with an online softmax so that the N x N score matrix never reaches
+ * device memory ("1-Flash-Attention.md", sections "Tiling（分块）技术" and
+ * "递归计算softmax"; FlashAttention V2 page: Q tiles in the outer loop, K/V in the
+ * inner loop, normalisation once at the end). Single-query decode splits the
+ * key range across thread blocks and merges the partial results by their
+ * log-sum-exp (FlashAttention V2 page, Flash-Decoding paragraph; FlashAttention-3
+ * page, the split-K combine step).
+ *
+ * Conventions shared by every call:
+ *  - All tensors are dense, contiguous, row-major device buffers owned by the
+ *    caller. The library allocates nothing, never synchronises, and only
+ *    enqueues work on `stream` (0 = the legacy default stream). Every call is
+ *    asynchronous like a kernel launch.
+ *  - bf16 buffers hold IEEE bfloat16 bit patterns; float buffers hold IEEE fp32.
+ *  - Every pointer must be 16-byte aligned and must not alias another argument.
+ *  - Arguments are checked before anything is launched; a failed check returns a
+ *    status and enqueues nothing. A launch failure returns ATTN_ERR_CUDA.
+ *  - Every wait inside a kernel is bounded. A kernel whose wait runs out records
+ *    ATTN_ERR_TIMEOUT in a device-side status word and returns early (its outputs
+ *    are then undefined); attn_device_status() reads and clears that word.
+ *  - LSE is the natural-log log-sum-exp of the scaled, masked scores of a row:
+ *    lse_i = ln sum_{j visible} exp(scale * q_i . k_j).
+ */
+#ifndef EXACT_ATTENTION_RING_B200_ATTN_H
+#define EXACT_ATTENTION_RING_B200_ATTN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as the CUDA runtime's cudaStream_t (an opaque driver stream). */
+typedef struct CUstream_st* attn_stream_t;
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, Hq % Hkv != 0, bad scale */
+    ATTN_ERR_UNSUPPORTED = 2, /* a head dimension other than 64 or 128 */
+    ATTN_ERR_CUDA = 3,        /* a CUDA runtime call or a launch failed */
+    ATTN_ERR_TIMEOUT = 4      /* a bounded in-kernel wait ran out (see attn_device_status) */
+} attn_status_t;
+
+/*
+ * attn_fwd — prefill forward pass.
+ * Defined by: "1-Flash-Attention.md", "问题分析" (S = Q K^T, A = softmax(S/sqrt(d)),
+ * O = A V on (batch, heads, seq_len, head_dim) tensors) and "使用注意事项"
+ * (causal flag; head_dim 64 or 128; fp16/bf16 inputs), computed by the tiled
+ * online-softmax recurrence of "递归计算softmax"; softmax_scale as in "框架集成".
+ *
+ *  q    [B, Hq,  N, d] bf16 (device, read)
+ *  k, v [B, Hkv, N, d] bf16 (device, read)
+ *  o    [B, Hq,  N, d] bf16 (device, written): O rounded to nearest-even bf16
+ *  lse  [B, Hq,  N]    fp32 (device, written): natural-log LSE per row
+ *  B, Hq, Hkv, N >= 1; Hq % Hkv == 0; query head h reads key/value head
+ *      h / (Hq / Hkv) (grouped-query / multi-query attention).
+ *  d     64 or 128 (else ATTN_ERR_UNSUPPORTED).
+ *  causal  0: every row sees all N keys; 1: row i sees keys j <= i.
+ *  scale   finite and > 0 (typically 1/sqrt(d)).
+ * Any N >= 1 is accepted (no power-of-two requirement); ragged tiles are masked.
+ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                       int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                       attn_stream_t stream);
+
+/*
+ * attn_decode_splitkv — split-KV (Flash-Decoding) partials for one query token.
+ * Defined by: FlashAttention V2 page, Flash-Decoding paragraph (the key/value
+ * sequence is split across thread blocks for single-query decode); each split is
+ * the attention of "1-Flash-Attention.md", "问题分析", restricted to its keys.
+ *
+ *  q        [B, Hq, d]      bf16 (device, read): the one query of each sequence
+ *  k, v     [B, Hkv, L, d]  bf16 (device, read): the key/value cache
+ *  o_part   [B, Hq, S, d]   fp32 (device, written): normalised partial outputs
+ *  lse_part [B, Hq, S]      fp32 (device, written): natural-log LSE per split
+ *  S = num_splits, 1 <= S <= L. Split s covers keys [s*C, min(L, (s+1)*C)) with
+ *  C = 32 * ceil(ceil(L / S) / 32). A split with no keys gets lse = -inf, o = 0.
+ *  d 64 or 128; Hq % Hkv == 0; scale finite and > 0.
+ */
+attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v,
+                                  float* o_part, float* lse_part,
+                                  int B, int Hq, int Hkv, int L, int d, int num_splits,
+                                  float scale, attn_stream_t stream);
+
+/*
+ * attn_combine — log-sum-exp weighted merge of split partials.
+ * Defined by: FlashAttention-3 page (the split-K combine step,
+ * combine_attn_seqk_parallel): with M = max_s lse_s and w_s = exp(lse_s - M),
+ * O = sum_s w_s O_s / sum_s w_s and LSE = M + ln sum_s w_s; a split with
+ * lse_s = -inf has weight 0.
+ *
+ *  o_part   [B, Hq, S, d] fp32 (device, read)
+ *  lse_part [B, Hq, S]    fp32 (device, read)
+ *  o        [B, Hq, d]    bf16 (device, written)
+ *  lse      [B, Hq]       fp32 (device, written)
+ *  d 64 or 128; S >= 1; at least one split of every (b, h) must be non-empty.
+ */
+attn_status_t attn_combine(const float* o_part, const float* lse_part, void* o, float* lse,
+                           int B, int Hq, int num_splits, int d, attn_stream_t stream);
+
+/*
+ * attn_decode_default_splits — the split count attn_decode_splitkv is tuned for:
+ * enough (batch, kv-head, split) blocks to fill every SM about twice, with at
+ * least 256 keys per split. Pure host arithmetic; returns >= 1, or 0 on bad args.
+ */
+int attn_decode_default_splits(int B, int Hq, int Hkv, int L);
+
+/* Human-readable name of a status code (static storage). */
+const char* attn_status_string(attn_status_t status);
+
+/*
+ * attn_device_status — synchronises `stream`, then reads and clears the
+ * device-side status word that kernels set when a bounded wait runs out.
+ * Returns ATTN_OK, ATTN_ERR_TIMEOUT, or ATTN_ERR_CUDA if synchronisation failed.
+ * Uses the current CUDA device.
+ */
+attn_status_t attn_device_status(attn_stream_t stream);
+
+/*
+ * attn_selftest_bounded_wait — launches one thread that waits on a barrier that
+ * nothing completes, with a wait limit of `limit_us` microseconds (1..10^6), so
+ * that the timeout path can be exercised without faulting or hanging the GPU.
+ * The wait runs out, the kernel records ATTN_ERR_TIMEOUT and returns. Enqueued
+ * on `stream`; read the result with attn_device_status().
+ */
+attn_status_t attn_selftest_bounded_wait(int limit_us, attn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTENTION_RING_B200_ATTN_H */

@@ -39,13 +39,20 @@ def make_qkv(seed: int, B: int, Hq: int, Hkv: int, N: int, d: int, q_mult: float
     return q.contiguous(), k.contiguous(), v.contiguous()
 
 
-def make_decode(seed: int, B: int, Hq: int, Hkv: int, L: int, d: int):
-    """Single-query decode inputs: q [B,Hq,d], k/v [B,Hkv,L,d], bf16 CPU tensors."""
+def make_decode(seed: int, B: int, Hq: int, Hkv: int, L: int, d: int, pin: bool = False):
+    """Single-query decode inputs: q [B,Hq,d], k/v [B,Hkv,L,d], bf16 CPU tensors.
+
+    Drawn in the order q, then k one batch entry at a time, then v likewise,
+    so that a large cache never needs a full float32 copy on the host.
+    """
     gen = torch.Generator().manual_seed(seed)
-    q = _randn_bf16(gen, (B, Hq, d))
-    k = _randn_bf16(gen, (B, Hkv, L, d))
-    v = _randn_bf16(gen, (B, Hkv, L, d))
-    return q.contiguous(), k.contiguous(), v.contiguous()
+    q = _randn_bf16(gen, (B, Hq, d)).contiguous()
+    k = torch.empty(B, Hkv, L, d, dtype=torch.bfloat16, pin_memory=pin)
+    v = torch.empty(B, Hkv, L, d, dtype=torch.bfloat16, pin_memory=pin)
+    for t in (k, v):
+        for b in range(B):
+            t[b] = _randn_bf16(gen, (Hkv, L, d))
+    return q, k, v
 
 
 def sample_rows(seed: int, B: int, H: int, N: int, tile: int = 128, per_slice: int = 256,

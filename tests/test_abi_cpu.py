@@ -1,0 +1,132 @@
+"""Host-side tests of the C ABI: no GPU needed, nothing is launched.
+
+The library must load, export every entry point include/attn.h declares, and
+reject bad arguments with the documented status before touching the device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_attention_ring_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(attn_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("attn_fwd", "attn_decode_splitkv", "attn_combine"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_names_match_the_abi():
+    import exact_attention_ring_b200 as eab
+    for n in declared_functions():
+        assert hasattr(eab, n), n
+
+
+def _fwd(lib, q=16, k=32, v=48, o=64, lse=80, B=1, Hq=2, Hkv=1, N=8, d=64, causal=0, scale=0.125):
+    P = ctypes.c_void_p
+    lib.attn_fwd.restype = ctypes.c_int
+    return lib.attn_fwd(P(q), P(k), P(v), P(o), P(lse), B, Hq, Hkv, N, d, causal, ctypes.c_float(scale), None)
+
+
+def _dec(lib, q=16, k=32, v=48, op=64, lp=80, B=1, Hq=4, Hkv=2, L=100, d=128, S=4, scale=0.1):
+    P = ctypes.c_void_p
+    lib.attn_decode_splitkv.restype = ctypes.c_int
+    return lib.attn_decode_splitkv(P(q), P(k), P(v), P(op), P(lp), B, Hq, Hkv, L, d, S, ctypes.c_float(scale), None)
+
+
+def _comb(lib, op=16, lp=32, o=48, lse=64, B=1, Hq=4, S=3, d=64):
+    P = ctypes.c_void_p
+    lib.attn_combine.restype = ctypes.c_int
+    return lib.attn_combine(P(op), P(lp), P(o), P(lse), B, Hq, S, d, None)
+
+
+INVALID, UNSUPPORTED = 1, 2
+
+
+@pytest.mark.parametrize("kw", [dict(q=0), dict(k=0), dict(v=0), dict(o=0), dict(lse=0), dict(q=17),
+                                dict(o=24), dict(B=0), dict(Hq=0), dict(Hkv=0), dict(N=0), dict(Hq=3, Hkv=2),
+                                dict(causal=2), dict(scale=0.0), dict(scale=-1.0), dict(scale=float("inf")),
+                                dict(scale=float("nan"))])
+def test_fwd_rejects_invalid(lib, kw):
+    assert _fwd(lib, **kw) == INVALID
+
+
+@pytest.mark.parametrize("d", [0, 8, 32, 96, 256])
+def test_fwd_rejects_unsupported_head_dim(lib, d):
+    assert _fwd(lib, d=d) == UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw", [dict(q=0), dict(op=0), dict(lp=8), dict(L=0), dict(S=0), dict(S=101),
+                                dict(Hq=5, Hkv=2), dict(scale=0.0), dict(B=0)])
+def test_decode_rejects_invalid(lib, kw):
+    assert _dec(lib, **kw) == INVALID
+
+
+def test_decode_rejects_unsupported_head_dim(lib):
+    assert _dec(lib, d=80) == UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw", [dict(op=0), dict(lse=4), dict(B=0), dict(Hq=0), dict(S=0)])
+def test_combine_rejects_invalid(lib, kw):
+    assert _comb(lib, **kw) == INVALID
+
+
+def test_combine_rejects_unsupported_head_dim(lib):
+    assert _comb(lib, d=100) == UNSUPPORTED
+
+
+def test_status_strings(lib):
+    lib.attn_status_string.restype = ctypes.c_char_p
+    names = [lib.attn_status_string(i).decode() for i in range(5)]
+    assert names == ["ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA",
+                     "ATTN_ERR_TIMEOUT"]
+    assert lib.attn_status_string(99).decode() == "ATTN_ERR_UNKNOWN"
+
+
+def test_selftest_rejects_bad_limit(lib):
+    lib.attn_selftest_bounded_wait.restype = ctypes.c_int
+    assert lib.attn_selftest_bounded_wait(0, None) == INVALID
+    assert lib.attn_selftest_bounded_wait(2_000_000, None) == INVALID
+
+
+def test_default_splits(lib):
+    f = lib.attn_decode_default_splits
+    f.restype = ctypes.c_int
+    assert f(0, 32, 8, 100) == 0 and f(1, 30, 8, 100) == 0
+    # B=1, 8 KV heads, 4 query heads each: 8 blocks per split; about 2 x 148 blocks wanted
+    assert f(1, 32, 8, 32768) == 37
+    assert f(1, 32, 8, 4096) == 16        # capped by >= 256 keys per split
+    assert f(8, 32, 8, 131072) == 5
+    assert f(1, 1, 1, 1) == 1
+    for L in (1, 31, 257, 100000):
+        s = f(2, 16, 4, L)
+        assert 1 <= s <= L
+
+
+def test_decode_chunk_rule():
+    from exact_attention_ring_b200 import decode_chunk
+    assert decode_chunk(4096, 16) == 256
+    assert decode_chunk(32768, 37) == 896
+    assert decode_chunk(100, 64) == 32
+    assert decode_chunk(1, 1) == 32
