@@ -19,6 +19,7 @@ from ._binding import (  # noqa: F401
     attention,
     attn_combine,
     attn_decode_default_splits,
+    attn_decode_noalloc,
     attn_decode_splitkv,
     attn_device_status,
     attn_fwd,

@@ -27,7 +27,7 @@ def _load():
     if not os.path.exists(_LIB_PATH):
         raise ImportError(
             f"exact_attention_ring_b200: CUDA library not built ({_LIB_PATH}); "
-            "run `python -m exact_attention_ring_b200.build`")
+            "run `python exact_attention_ring_b200/build.py`")
     lib = ctypes.CDLL(_LIB_PATH)
     P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
@@ -44,6 +44,8 @@ def _load():
     lib.attn_device_status.restype = I
     lib.attn_selftest_bounded_wait.argtypes = [I, P]
     lib.attn_selftest_bounded_wait.restype = I
+    lib.attn_decode_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.attn_decode_noalloc.restype = I
     return lib
 
 
@@ -169,3 +171,18 @@ def decode(q, k, v, scale: float | None = None, num_splits: int | None = None, s
     lse = torch.empty(B, Hq, device=q.device, dtype=torch.float32)
     attn_combine(o_part, lse_part, o, lse, stream)
     return o, lse
+
+
+def attn_decode_noalloc(q, k, v, o, lse, num_splits: int, scale: float, stream=None):
+    """Decode plus combine with the partials in the library's fixed device array
+    (no allocation anywhere). q [B,Hq,d], k/v [B,Hkv,L,d] bf16 -> o [B,Hq,d] bf16,
+    lse [B,Hq] fp32. Needs B*Hq*num_splits*(d+1) <= 1,048,576."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, torch.bfloat16, n)
+    _need(lse, torch.float32, "lse")
+    B, Hq, d = q.shape
+    Hkv, L = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, L, d) or v.shape != k.shape or o.shape != (B, Hq, d) or lse.shape != (B, Hq):
+        raise ValueError("attn_decode_noalloc: inconsistent shapes")
+    _check(_lib.attn_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, L, d,
+                                    int(num_splits), float(scale), _stream(stream)), "attn_decode_noalloc")

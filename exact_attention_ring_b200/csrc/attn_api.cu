@@ -213,3 +213,63 @@ attn_status_t attn_selftest_bounded_wait(int limit_us, attn_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without any device allocation by the caller or the library.
+//
+// Some callers cannot hand this library a scratch buffer for the split
+// partials: code that runs where the device memory is already fully owned by
+// another allocator (a serving engine's pre-reserved pool, a host application
+// that forbids allocations from plug-ins), or latency-critical loops where a
+// cudaMalloc and the device synchronisation it can imply are not acceptable.
+// For them, attn_decode_noalloc keeps the partials in one fixed array compiled
+// into the library: a file-scope __device__ array that every GPU which loads the
+// library holds until the process exits.
+namespace eab {
+namespace {
+
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;  // 4 MiB per device
+static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchFloats];
+
+// Host code only holds a stand-in for the array's name; the device address is
+// looked up once per device (with that device current) and cached.
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+attn_status_t scratch_for_current_device(float** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || ptr == nullptr) return ATTN_ERR_CUDA;
+        g_scratch_ptr[dev] = ptr;
+    }
+    *out = static_cast<float*>(g_scratch_ptr[dev]);
+    return ATTN_OK;
+}
+
+}  // namespace
+}  // namespace eab
+
+extern "C" attn_status_t attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                                             int B, int Hq, int Hkv, int L, int d, int num_splits, float scale,
+                                             attn_stream_t stream) {
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return ATTN_ERR_INVALID_ARG;
+    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || num_splits < 1 || num_splits > L) return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    // partials: o_part [B,Hq,S,d] then lse_part [B,Hq,S], all fp32
+    const unsigned long long units = static_cast<unsigned long long>(B) * Hq * num_splits;
+    if (units * (static_cast<unsigned long long>(d) + 1) > kNoAllocScratchFloats) return ATTN_ERR_INVALID_ARG;
+    float* scratch = nullptr;
+    if (attn_status_t st = scratch_for_current_device(&scratch); st != ATTN_OK) return st;
+    float* o_part = scratch;
+    float* lse_part = scratch + units * d;  // d*4 bytes per unit keeps this 16-byte aligned
+    if (attn_status_t st = attn_decode_splitkv(q, k, v, o_part, lse_part, B, Hq, Hkv, L, d, num_splits, scale,
+                                               stream);
+        st != ATTN_OK)
+        return st;
+    return attn_combine(o_part, lse_part, o, lse, B, Hq, num_splits, d, stream);
+}

@@ -127,6 +127,34 @@ attn_status_t attn_device_status(attn_stream_t stream);
  */
 attn_status_t attn_selftest_bounded_wait(int limit_us, attn_stream_t stream);
 
+/*
+ * attn_decode_noalloc — split-KV decode plus combine that allocates nothing.
+ * The pages have no counterpart: this is a service for callers that cannot
+ * allocate device memory for the split partials (an engine whose device memory
+ * is owned by its own pool, a plug-in that must not allocate, a latency-critical
+ * loop that cannot afford cudaMalloc). It computes what attn_decode_splitkv
+ * followed by attn_combine computes, with the same arguments except that the
+ * partials live in a fixed 4 MiB array built into the library (1,048,576 floats;
+ * every GPU that loads the library holds it until the process exits).
+ *
+ *  q [B, Hq, d], k/v [B, Hkv, L, d] bf16 (device, read)
+ *  o [B, Hq, d] bf16, lse [B, Hq] fp32 (device, written)
+ *  num_splits, d, scale: as for attn_decode_splitkv.
+ * Limit: B * Hq * num_splits * (d + 1) <= 1,048,576; larger problems return
+ * ATTN_ERR_INVALID_ARG before anything is enqueued (use fewer splits, or the
+ * attn_decode_splitkv + attn_combine pair with caller-owned partials).
+ * The first call on a device looks up the array's device address once (with
+ * that device current); make that first call before any stream capture.
+ * The call never calls cudaMalloc, cudaFree or any allocating routine. All calls
+ * on a device share the one array and it keeps the last call's contents;
+ * nothing in it needs clearing, because every partial is written before it is
+ * read. Calls that can overlap on the GPU (different streams without ordering
+ * between them) race on the array and must not be issued.
+ */
+attn_status_t attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                                  int B, int Hq, int Hkv, int L, int d, int num_splits, float scale,
+                                  attn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
