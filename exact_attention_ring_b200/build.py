@@ -1,6 +1,6 @@
 """Builds the sm_100a CUDA library (csrc/attn_api.cu, one translation unit) in-tree.
 
-    python -m exact_attention_ring_b200.build [--force] [--verbose]
+    python exact_attention_ring_b200/build.py [--force] [--verbose]
 
 produces exact_attention_ring_b200/_lib/libattn_b200.so with nvcc
 ``-gencode arch=compute_100a,code=sm_100a``. The CUDA runtime is linked

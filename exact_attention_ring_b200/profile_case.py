@@ -1,0 +1,64 @@
+"""Runs one kernel of the library a few times on seeded inputs, for profilers.
+
+    python -m exact_attention_ring_b200.profile_case fwd --B 4 --H 32 --N 2048 --d 128 --causal 1 --iters 3
+    python -m exact_attention_ring_b200.profile_case decode --B 1 --H 32 --Hkv 8 --L 131072 --d 128 --iters 3
+
+Meant to be wrapped by ncu (one kernel, a few launches, inputs larger than L2
+but a few GB at most). Prints the CUDA-event time of the last launch.
+"""
+import argparse
+import os
+import sys
+
+import torch
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+
+import exact_attention_ring_b200 as eab  # noqa: E402
+import seeded_inputs as si  # noqa: E402
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("kernel", choices=["fwd", "decode"])
+    ap.add_argument("--B", type=int, default=4)
+    ap.add_argument("--H", type=int, default=32)
+    ap.add_argument("--Hkv", type=int, default=0)
+    ap.add_argument("--N", type=int, default=2048)
+    ap.add_argument("--L", type=int, default=131072)
+    ap.add_argument("--d", type=int, default=128)
+    ap.add_argument("--causal", type=int, default=1)
+    ap.add_argument("--iters", type=int, default=3)
+    a = ap.parse_args()
+    Hkv = a.Hkv or a.H
+    dev = torch.device("cuda", 0)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if a.kernel == "fwd":
+        q, k, v = (t.to(dev) for t in si.make_qkv(1001, a.B, a.H, Hkv, a.N, a.d))
+        o = torch.empty_like(q)
+        lse = torch.empty(a.B, a.H, a.N, device=dev)
+        for _ in range(a.iters):
+            start.record()
+            eab.attn_fwd(q, k, v, o, lse, bool(a.causal), a.d ** -0.5)
+            end.record()
+        flops = 4.0 * a.B * a.H * a.N * a.N * a.d / (2 if a.causal else 1)
+    else:
+        q, k, v = (t.to(dev) for t in si.make_decode(1004, a.B, a.H, Hkv, a.L, a.d))
+        S = eab.attn_decode_default_splits(a.B, a.H, Hkv, a.L)
+        o_part = torch.empty(a.B, a.H, S, a.d, device=dev)
+        lse_part = torch.empty(a.B, a.H, S, device=dev)
+        for _ in range(a.iters):
+            start.record()
+            eab.attn_decode_splitkv(q, k, v, o_part, lse_part, S, a.d ** -0.5)
+            end.record()
+        flops = 2.0 * a.B * Hkv * a.L * a.d * 2  # bytes for decode
+    torch.cuda.synchronize()
+    assert eab.attn_device_status() == 0
+    ms = start.elapsed_time(end)
+    unit = "TFLOPS" if a.kernel == "fwd" else "GB/s"
+    val = flops / (ms * 1e-3) / (1e12 if a.kernel == "fwd" else 1e9)
+    print(f"{a.kernel}: {ms:.4f} ms  {val:.1f} {unit}")
+
+
+if __name__ == "__main__":
+    main()

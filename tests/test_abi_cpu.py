@@ -15,9 +15,11 @@ HEADER = os.path.join(ROOT, "include", "attn.h")
 
 @pytest.fixture(scope="module")
 def lib():
-    from exact_attention_ring_b200 import build
-    path = build.build()
-    return ctypes.CDLL(path)
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("eab_build", os.path.join(ROOT, "exact_attention_ring_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
+    return ctypes.CDLL(build.build())
 
 
 def declared_functions():
