@@ -63,7 +63,7 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     auto kern = attn_fwd_kernel<D, CAUSAL>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
-    const long long grid = static_cast<long long>(p.n_qtiles) * p.B * p.Hq;
+    const long long grid = static_cast<long long>(p.n_qblocks) * p.B * p.Hq;
     if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
     kern<<<static_cast<unsigned>(grid), C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -136,7 +136,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N;
-    p.n_qtiles = (N + 127) / 128;
+    p.n_qblocks = (N + 255) / 256;
     p.scale_log2 = scale * kLog2e;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d == 128) return causal ? launch_fwd<128, true>(tq, tk, tv, p, st) : launch_fwd<128, false>(tq, tk, tv, p, st);

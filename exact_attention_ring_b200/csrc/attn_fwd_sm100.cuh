@@ -1,27 +1,36 @@
 // Prefill forward pass on sm_100a: O = softmax(scale * Q K^T) V and the per-row
-// log-sum-exp, one 128-row query tile per CTA.
+// log-sum-exp.
 //
 // The method is the tiled online softmax of "1-Flash-Attention.md" (sections
 // "Tiling（分块）技术", "递归计算softmax"): a query tile stays on chip while key /
 // value tiles stream past it; per row a running max m and denominator l are
 // kept, the accumulator is rescaled when the max moves, and O is divided by l
 // once at the end (FlashAttention V2 page: fewer non-matmul operations). Loop
-// order is the V2 one (query tile outer, key/value tiles inner).
+// order is the V2 one (query tiles outer, key/value tiles inner).
 //
-// B200 mapping (warp-specialised, 192 threads):
-//   warp 0    TMA producer: the Q tile once, then K_j and V_j tiles into a ring
-//             of shared-memory slots guarded by full/empty mbarriers.
-//   warp 1    MMA issuer (one thread): S_j = Q K_j^T with tcgen05.mma into one of
-//             two TMEM score buffers, and O += P_j V_j with P read from TMEM.
-//             Completion is signalled with tcgen05.commit onto mbarriers.
-//   warps 2-5 softmax: one thread per query row (TMEM lane). Reads S_j, applies
-//             the causal / ragged-tail mask, tracks the running max in log2
-//             units (exp2 with scale*log2(e) folded into one FMA), rescales O in
-//             TMEM only when the max grows by more than 2^8 (lazy rescale), writes
-//             P_j as bf16 over the S_j columns, and finally normalises O.
-// TMEM columns: S buffer 0 [0,128), S buffer 1 [128,256), O [256, 256+D).
-// Shared memory: Q tile + SLOTS key/value tiles, all 128-byte swizzled as the
-// tcgen05 K-major (Q, K) and MN-major (V) operand layouts expect.
+// B200 mapping. One CTA owns two 128-row query tiles of one head (256 rows)
+// that share every K/V tile; 384 threads, warp-specialised:
+//   warps 0-3   softmax of query tile 0, one thread per row (TMEM lane);
+//   warps 4-7   softmax of query tile 1;
+//   warp 8, 9   MMA issuers, one per query tile. A thread that has just issued
+//               tcgen05.mma cannot act on an mbarrier for several hundred cycles,
+//               so two issuing warps keep the tensor core busy while each waits;
+//   warps 10,11 TMA producers: the two Q tiles, then K_j and V_j into a ring of
+//               shared-memory slots (full/empty mbarriers). One issuing thread
+//               streams TMA boxes one after another, so the boxes of every tile
+//               are split between two threads.
+// Per query tile t and key tile j:
+//   S_t = Q_t K_j^T           tcgen05.mma (A, B K-major in smem) -> TMEM S_t;
+//   softmax                   pass 1 reads S_t and takes the row max; when it has
+//                             grown by more than 2^8 (log2 units) O_t is rescaled
+//                             in TMEM (lazy rescale); pass 2 computes
+//                             p = exp2(s*scale*log2e - m) with one FMA, sums l in
+//                             fp32 and writes P_t as bf16 over the S_t columns;
+//   O_t += P_t V_j            tcgen05.mma with A = P_t from TMEM, B = V_j MN-major;
+// S_t(j+1) is issued after O_t += P_t(j) V_j by the same thread, so the tensor
+// pipe's issue order keeps P_t(j) intact until it has been read, and S_t(j+1)'s
+// completion implies that O_t holds every earlier P V product.
+// TMEM columns: tile t uses S [256t, 256t+128) and O [256t+128, 256t+128+D).
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -32,28 +41,43 @@ struct FwdParams {
     __nv_bfloat16* o;  // [B, Hq, N, D]
     float* lse;        // [B, Hq, N]
     int B, Hq, Hkv, N;
-    int n_qtiles;
+    int n_qblocks;     // ceil(N / 256)
     float scale_log2;  // scale * log2(e)
 };
 
 template <int D>
 struct FwdCfg {
-    static constexpr int BM = 128;                 // query rows per tile (= TMEM lanes)
-    static constexpr int BN = 128;                 // keys per tile
+    static constexpr int BM = 128;                 // rows per query tile (= TMEM lanes)
+    static constexpr int TILES = 2;                // query tiles per CTA
+    static constexpr int BN = 128;                 // keys per K/V tile
     static constexpr int CHUNKS = D / 64;          // 64-element (128-byte) swizzle chunks per row
-    static constexpr int Q_BYTES = BM * D * 2;
+    static constexpr int Q_TILE_BYTES = BM * D * 2;
     static constexpr int TILE_BYTES = BN * D * 2;  // one K or V tile
-    static constexpr int SLOTS = (D == 128) ? 6 : 10;
-    static constexpr int NUM_THREADS = 192;
-    static constexpr int NUM_BARRIERS = 1 + 2 * SLOTS + 2 + 2 + 1 + 1;
-    static constexpr int SMEM_BYTES = 1024 + Q_BYTES + SLOTS * TILE_BYTES + NUM_BARRIERS * 8 + 16;
+    static constexpr int SLOTS = (D == 128) ? 5 : 10;
+    static constexpr int NUM_THREADS = 384;
+    static constexpr int NUM_PRODUCERS = 2;
+    static constexpr int NUM_BARRIERS = 2 + 2 * SLOTS + 2 + 2 + 2 + 2;
+    static constexpr int SMEM_BYTES = 1024 + TILES * Q_TILE_BYTES + SLOTS * TILE_BYTES + NUM_BARRIERS * 8 + 16;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t O_COL = 256;
     static constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: P <= 2^8 between rescales
 };
 
+// Max of 64 values with eight independent chains of 3-input max.
+__device__ __forceinline__ float max64(const float (&v)[64]) {
+    float m[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m[k] = max3(v[k], v[8 + k], v[16 + k]);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m[k] = max3(m[k], v[24 + k], v[32 + k]);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m[k] = max3(m[k], v[40 + k], v[48 + k]);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m[k] = fmaxf(m[k], v[56 + k]);
+    return max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
     using C = FwdCfg<D>;
@@ -61,46 +85,48 @@ __global__ void __launch_bounds__(192, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
-    uint8_t* sKV = smem + C::Q_BYTES;
+    uint8_t* sKV = smem + C::TILES * C::Q_TILE_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + SLOTS * C::TILE_BYTES);
-    uint64_t* q_full = bars;
-    uint64_t* slot_full = bars + 1;
-    uint64_t* slot_empty = slot_full + SLOTS;
-    uint64_t* s_full = slot_empty + SLOTS;  // [2]
-    uint64_t* p_full = s_full + 2;          // [2]
-    uint64_t* o_done = p_full + 2;
-    uint64_t* drain = o_done + 1;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* q_full = bars;                   // [2]
+    uint64_t* slot_full = q_full + 2;          // [SLOTS]
+    uint64_t* slot_empty = slot_full + SLOTS;  // [SLOTS]
+    uint64_t* s_full = slot_empty + SLOTS;     // [2]
+    uint64_t* p_full = s_full + 2;             // [2]
+    uint64_t* o_done = p_full + 2;             // [2]
+    uint64_t* drain = o_done + 2;              // [2]
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // Work tile: heaviest causal query tiles are scheduled first.
+    // Work: one 256-row query block of one (batch, head); heaviest causal blocks first.
     const int bh_count = p.B * p.Hq;
     const int rank = blockIdx.x / bh_count;
     const int bh = blockIdx.x % bh_count;
-    const int qt = CAUSAL ? (p.n_qtiles - 1 - rank) : rank;
+    const int qb = CAUSAL ? (p.n_qblocks - 1 - rank) : rank;
     const int b = bh / p.Hq, h = bh % p.Hq;
     const int hk = h / (p.Hq / p.Hkv);
-    const int n_kv_tiles = (p.N + BN - 1) / BN;
-    const int nk = CAUSAL ? min(qt + 1, n_kv_tiles) : n_kv_tiles;
+    const int n_kv = (p.N + BN - 1) / BN;
+    // key tiles each query tile needs (tile 1 needs at most one more than tile 0)
+    const int nk0 = CAUSAL ? min(2 * qb + 1, n_kv) : n_kv;
+    const int nk1 = CAUSAL ? min(2 * qb + 2, n_kv) : n_kv;
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&q_full[t], C::CHUNKS);  // one expect_tx arrival per box
+            mbar_init(&s_full[t], 1);
+            mbar_init(&p_full[t], 128);
+            mbar_init(&o_done[t], 1);
+            mbar_init(&drain[t], 1);
+        }
         for (int i = 0; i < SLOTS; ++i) {
-            mbar_init(&slot_full[i], 1);
-            mbar_init(&slot_empty[i], 1);
+            mbar_init(&slot_full[i], C::CHUNKS);
+            mbar_init(&slot_empty[i], 2);  // released by both query tiles' MMAs
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 128);
-        }
-        mbar_init(o_done, 1);
-        mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == 8) {
         tmem_alloc(tmem_holder, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -109,118 +135,140 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    if (warp == 0) {
-        // ------------------------------------------------------ producer ----
+    if (warp >= 10) {
+        // ------------------------------------------------------ producers ---
+        // Box c of Q tile t, and box c of item i (K_j = item 2j, V_j = item
+        // 2j+1), go to producer (index * CHUNKS + c) % 2; each box arrives on its
+        // full barrier with its own byte count.
         if (lane == 0) {
+            const int me = warp - 10;
             const int zq = b * p.Hq + h, zkv = b * p.Hkv + hk;
+            constexpr uint32_t BOX_BYTES = BN * 128;
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            mbar_arrive_expect_tx(q_full, C::Q_BYTES);
 #pragma unroll
-            for (int c = 0; c < C::CHUNKS; ++c) tma_load_3d(sQ + c * BM * 128, &tm_q, q_full, c * 64, qt * BM, zq);
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int c = 0; c < C::CHUNKS; ++c) {
+                    if ((t * C::CHUNKS + c) % C::NUM_PRODUCERS != me) continue;
+                    mbar_arrive_expect_tx(&q_full[t], BM * 128);
+                    tma_load_3d(sQ + t * C::Q_TILE_BYTES + c * BM * 128, &tm_q, &q_full[t], c * 64,
+                                qb * 2 * BM + t * BM, zq);
+                }
             int issued = 0;
-            for (int i = 0; i < 2 * nk; ++i) {
+            for (int i = 0; i < 2 * nk1; ++i) {
+                bool mine = false;
+#pragma unroll
+                for (int c = 0; c < C::CHUNKS; ++c) mine |= ((i * C::CHUNKS + c) % C::NUM_PRODUCERS) == me;
+                if (!mine) continue;
                 const int slot = i % SLOTS, use = i / SLOTS;
                 if (use > 0 && !mbar_wait(&slot_empty[slot], (use - 1) & 1, abort_flag)) break;
                 const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;
                 uint8_t* dst = sKV + slot * C::TILE_BYTES;
-                mbar_arrive_expect_tx(&slot_full[slot], C::TILE_BYTES);
 #pragma unroll
-                for (int c = 0; c < C::CHUNKS; ++c)
-                    tma_load_3d(dst + c * BN * 128, tm, &slot_full[slot], c * 64, (i >> 1) * BN, zkv);
+                for (int c = 0; c < C::CHUNKS; ++c) {
+                    if ((i * C::CHUNKS + c) % C::NUM_PRODUCERS != me) continue;
+                    mbar_arrive_expect_tx(&slot_full[slot], BOX_BYTES);
+                    tma_load_3d(dst + c * BOX_BYTES, tm, &slot_full[slot], c * 64, (i >> 1) * BN, zkv);
+                }
                 issued = i + 1;
             }
             // Let every copy in flight land before the CTA can exit.
-            mbar_wait(q_full, 0, nullptr);
+            mbar_wait(&q_full[0], 0, nullptr);
+            mbar_wait(&q_full[1], 0, nullptr);
             for (int i = max(0, issued - SLOTS); i < issued; ++i)
                 mbar_wait(&slot_full[i % SLOTS], (i / SLOTS) & 1, nullptr);
         }
-    } else if (warp == 1) {
-        // ---------------------------------------------------------- MMA -----
+    } else if (warp >= 8) {
+        // ---------------------------------------------------- MMA issuers ---
+        const int t = warp - 8;
         if (lane == 0) {
             constexpr uint32_t idesc_qk = make_idesc_bf16(BM, BN, 0, 0);
             constexpr uint32_t idesc_pv = make_idesc_bf16(BM, D, 0, 1);
-            const uint32_t q_addr = smem_addr(sQ), kv_addr = smem_addr(sKV);
-            bool ok = mbar_wait(q_full, 0, abort_flag);
-            auto issue_s = [&](int j) -> bool {
-                const int i = 2 * j, slot = i % SLOTS;
-                if (!mbar_wait(&slot_full[slot], (i / SLOTS) & 1, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t k_addr = kv_addr + slot * C::TILE_BYTES;
-                const uint32_t d_tmem = tmem + (j & 1) * 128;
+            const int nk = t ? nk1 : nk0;
+            const uint32_t s_tmem = tmem + t * 256, o_tmem = s_tmem + 128;
+            const uint32_t q_addr = smem_addr(sQ + t * C::Q_TILE_BYTES), kv_addr = smem_addr(sKV);
+            // item i (K_j = 2j, V_j = 2j+1) sits in slot i % SLOTS, use i / SLOTS
+            bool ok = mbar_wait(&q_full[t], 0, abort_flag) && mbar_wait(&slot_full[0], 0, abort_flag);
+            for (int j = 0; ok && j <= nk; ++j) {
+                if (j > 0) {
+                    // O_t += P_t(j-1) V_{j-1}; everything it and S_t(j) need is
+                    // awaited first so that both groups go out back to back.
+                    const int iv = 2 * j - 1, ik = 2 * j;
+                    ok = mbar_wait(&p_full[t], (j - 1) & 1, abort_flag) &&
+                         mbar_wait(&slot_full[iv % SLOTS], (iv / SLOTS) & 1, abort_flag) &&
+                         (j >= nk || mbar_wait(&slot_full[ik % SLOTS], (ik / SLOTS) & 1, abort_flag));
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t v_addr = kv_addr + (iv % SLOTS) * C::TILE_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk) {
+                        // V as the MN-major B operand: 16 keys = 2048 bytes per step;
+                        // LBO = distance between the 64-column chunks of the tile.
+                        const uint64_t bd = make_sdesc_sw128(v_addr + kk * 16 * 128, BN * 128, 1024);
+                        mma_ts(o_tmem, s_tmem + kk * 8, bd, idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&o_done[t]);
+                    if (t == 1 && j - 1 >= nk0) mbar_arrive(&slot_empty[iv % SLOTS]);  // tile-1-only item
+                    tc_commit(&slot_empty[iv % SLOTS]);
+                    if (j >= nk) break;
+                } else {
+                    tc_fence_after();
+                }
+                // S_t(j) = Q_t K_j^T
+                const int ik = 2 * j;
+                const uint32_t k_addr = kv_addr + (ik % SLOTS) * C::TILE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk & 3) * 32;  // 16 elements = 32 bytes inside the swizzle row
-                    const uint64_t ad = make_sdesc_sw128(q_addr + (kk >> 2) * BM * 128 + koff, 16, 1024);
-                    const uint64_t bd = make_sdesc_sw128(k_addr + (kk >> 2) * BN * 128 + koff, 16, 1024);
-                    mma_ss(d_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint64_t ad = make_sdesc_sw128(q_addr + (kk >> 2) * (BM * 128) + koff, 16, 1024);
+                    const uint64_t bd = make_sdesc_sw128(k_addr + (kk >> 2) * (BN * 128) + koff, 16, 1024);
+                    mma_ss(s_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                tc_commit(&s_full[j & 1]);
-                tc_commit(&slot_empty[slot]);
-                return true;
-            };
-            if (ok) ok = issue_s(0);
-            if (ok && nk > 1) ok = issue_s(1);
-            for (int j = 0; ok && j < nk; ++j) {
-                if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag)) break;
-                const int i = 2 * j + 1, slot = i % SLOTS;
-                if (!mbar_wait(&slot_full[slot], (i / SLOTS) & 1, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t v_addr = kv_addr + slot * C::TILE_BYTES;
-                const uint32_t a_tmem = tmem + (j & 1) * 128;
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    // V tile as the MN-major B operand: 16 keys = 2048 bytes per step;
-                    // LBO = distance between the 64-column chunks of the tile.
-                    const uint64_t bd = make_sdesc_sw128(v_addr + kk * 16 * 128, BN * 128, 1024);
-                    mma_ts(tmem + C::O_COL, a_tmem + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                tc_commit(o_done);
-                tc_commit(&slot_empty[slot]);
-                if (j + 2 < nk) ok = issue_s(j + 2);
+                tc_commit(&s_full[t]);
+                if (t == 1 && j >= nk0) mbar_arrive(&slot_empty[ik % SLOTS]);  // tile-1-only item
+                tc_commit(&slot_empty[ik % SLOTS]);
             }
             // Every MMA must be complete before TMEM is released.
-            tc_commit(drain);
-            mbar_wait(drain, 0, nullptr);
+            tc_commit(&drain[t]);
+            mbar_wait(&drain[t], 0, nullptr);
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------ softmax -----
+        // ------------------------------------------------------- softmax ----
+        const int t = warp >> 2;
         const int quad = warp & 3;  // TMEM lane quadrant this warp may access
         const int row = quad * 32 + lane;
-        const int grow = qt * BM + row;
-        const uint32_t lane_base = tmem + (uint32_t(quad * 32) << 16);
+        const int grow = qb * 2 * BM + t * BM + row;
+        const int q128 = 2 * qb + t;  // index of this query tile in 128-row units
+        const int nk = t ? nk1 : nk0;
+        const uint32_t s_addr = tmem + t * 256 + (uint32_t(quad * 32) << 16);
+        const uint32_t o_addr = s_addr + 128;
         const float c2 = p.scale_log2;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nk; ++j) {
-            const bool w = mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag);
+            const bool w = mbar_wait(&s_full[t], j & 1, abort_flag);
             if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t s_addr = lane_base + (j & 1) * 128;
-            float s[BN];
+            // valid key columns of this tile for this row: [0, lim)
+            int lim = BN;
+            if (CAUSAL && j == q128) lim = row + 1;
+            if (!CAUSAL && j * BN + BN > p.N) lim = p.N - j * BN;
+            // pass 1: row max
+            float mx = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(s_addr + c * 32, r);
+            for (int half = 0; half < 2; ++half) {
+                uint32_t r[64];
+                tmem_ld64(s_addr + half * 64, r);
+                if (__any_sync(0xffffffffu, half * 64 + 64 > lim)) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+                    for (int i = 0; i < 64; ++i)
+                        if (half * 64 + i >= lim) r[i] = 0xff800000u;  // -inf
+                }
+                mx = fmaxf(mx, max64(reinterpret_cast<const float(&)[64]>(r)));
             }
-            const int kv0 = j * BN;
-            if (CAUSAL && j == qt) {
-#pragma unroll
-                for (int i = 0; i < BN; ++i)
-                    if (i > row) s[i] = -INFINITY;
-            } else if (!CAUSAL && kv0 + BN > p.N) {
-                const int lim = p.N - kv0;
-#pragma unroll
-                for (int i = 0; i < BN; ++i)
-                    if (i >= lim) s[i] = -INFINITY;
-            }
-            float mx = s[0];
-#pragma unroll
-            for (int i = 1; i < BN; ++i) mx = fmaxf(mx, s[i]);
             const float m_tile = mx * c2;
             const bool need = m_tile > m_used + C::RESCALE_THRESHOLD;
             float factor = 1.f;
@@ -229,48 +277,56 @@ __global__ void __launch_bounds__(192, 1)
                 m_used = m_tile;
             }
             l *= factor;
-            const float neg_m = -m_used;
-            float rs = 0.f;
-            uint32_t pk[BN / 2];
+            // S_t(j) completing implies O_t already holds every earlier P V
+            // product, so O_t can be rescaled now, before P_t(j) is released.
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
-            for (int i = 0; i < BN / 2; ++i) {
-                const float p0 = ex2_approx(fmaf(s[2 * i], c2, neg_m));
-                const float p1 = ex2_approx(fmaf(s[2 * i + 1], c2, neg_m));
-                rs += p0 + p1;
-                pk[i] = pack_bf16x2(p0, p1);
-            }
-            l += rs;
-            if (j > 0) {
-                // Every PV completion is awaited in order, so the parity wait on
-                // o_done can never alias a phase two completions back. PV_{j-1}
-                // was issued a whole tile ago, so this rarely stalls.
-                const bool w2 = mbar_wait(o_done, (j - 1) & 1, abort_flag);
-                if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
-                if (__any_sync(0xffffffffu, need)) {
-                    tc_fence_after();
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(o_addr + c * 32, r);
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t r[32];
-                        tmem_ld32(lane_base + C::O_COL + c * 32, r);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * factor);
-                        tmem_st32(lane_base + C::O_COL + c * 32, r);
-                    }
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * factor);
+                    tmem_st32(o_addr + c * 32, r);
                 }
             }
+            // pass 2: p = exp2(s * c2 - m), l += sum p, P (bf16) over the S columns.
+            // Rows of a tile with no masked column (every warp of a non-diagonal,
+            // non-tail tile) take a path with no per-element selects.
+            const bool full = __all_sync(0xffffffffu, lim == BN);
+            const float2 c2x2 = make_float2(c2, c2), negm2 = make_float2(-m_used, -m_used);
+            float2 rsum[4];
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c) {
-                uint32_t chunk[32];
+            for (int k = 0; k < 4; ++k) rsum[k] = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) chunk[i] = pk[c * 32 + i];
-                tmem_st32(s_addr + c * 32, chunk);
+            for (int half = 0; half < 2; ++half) {
+                uint32_t r[64];
+                tmem_ld64(s_addr + half * 64, r);
+                if (!full) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        if (half * 64 + i >= lim) r[i] = 0xff800000u;  // -inf: exp2 gives 0
+                }
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float2 y = ffma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
+                                           c2x2, negm2);
+                    const float2 pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+                    rsum[i & 3] = fadd2(rsum[i & 3], pp);
+                    pk[i] = pack_bf16x2(pp.x, pp.y);
+                }
+                tmem_st32(s_addr + half * 32, pk);
             }
+            const float2 rs = fadd2(fadd2(rsum[0], rsum[1]), fadd2(rsum[2], rsum[3]));
+            l += rs.x + rs.y;
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&p_full[j & 1]);
+            mbar_arrive(&p_full[t]);
         }
         if (ok) {
-            const bool w = mbar_wait(o_done, (nk - 1) & 1, abort_flag);
+            // PV(nk-2) is complete (S(nk-1) was seen), so the barrier is at most
+            // one phase away and this parity wait is exact.
+            const bool w = mbar_wait(&o_done[t], (nk - 1) & 1, abort_flag);
             if (__all_sync(0xffffffffu, w)) {
                 tc_fence_after();
                 const float inv_l = 1.f / l;
@@ -278,7 +334,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t r[32];
-                    tmem_ld32(lane_base + C::O_COL + c * 32, r);
+                    tmem_ld32(o_addr + c * 32, r);
                     uint32_t pk[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
@@ -298,7 +354,7 @@ __global__ void __launch_bounds__(192, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
