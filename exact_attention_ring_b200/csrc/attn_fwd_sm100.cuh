@@ -56,7 +56,7 @@ struct FwdCfg {
     static constexpr int SLOTS = (D == 128) ? 5 : 10;
     static constexpr int NUM_THREADS = 384;
     static constexpr int NUM_PRODUCERS = 2;
-    static constexpr int NUM_BARRIERS = 2 + 2 * SLOTS + 2 + 2 + 2 + 2;
+    static constexpr int NUM_BARRIERS = 2 + 2 * SLOTS + 2 + 2 + 2 + 2 + 2;
     static constexpr int SMEM_BYTES = 1024 + TILES * Q_TILE_BYTES + SLOTS * TILE_BYTES + NUM_BARRIERS * 8 + 16;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: P <= 2^8 between rescales
@@ -94,7 +94,8 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* p_full = s_full + 2;             // [2]
     uint64_t* o_done = p_full + 2;             // [2]
     uint64_t* drain = o_done + 2;              // [2]
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
+    uint64_t* turn = drain + 2;                // [2] softmax ping-pong
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(turn + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -115,9 +116,10 @@ __global__ void __launch_bounds__(384, 1)
         for (int t = 0; t < 2; ++t) {
             mbar_init(&q_full[t], C::CHUNKS);  // one expect_tx arrival per box
             mbar_init(&s_full[t], 1);
-            mbar_init(&p_full[t], 128);
+            mbar_init(&p_full[t], 4);  // one arrival per softmax warp
             mbar_init(&o_done[t], 1);
             mbar_init(&drain[t], 1);
+            mbar_init(&turn[t], 4);
         }
         for (int i = 0; i < SLOTS; ++i) {
             mbar_init(&slot_full[i], C::CHUNKS);
@@ -196,9 +198,11 @@ __global__ void __launch_bounds__(384, 1)
                     // O_t += P_t(j-1) V_{j-1}; everything it and S_t(j) need is
                     // awaited first so that both groups go out back to back.
                     const int iv = 2 * j - 1, ik = 2 * j;
-                    ok = mbar_wait(&p_full[t], (j - 1) & 1, abort_flag) &&
-                         mbar_wait(&slot_full[iv % SLOTS], (iv / SLOTS) & 1, abort_flag) &&
-                         (j >= nk || mbar_wait(&slot_full[ik % SLOTS], (ik / SLOTS) & 1, abort_flag));
+                    // (the loads are usually long complete: check them first so
+                    // that only the wait for P sits on the critical path)
+                    ok = mbar_wait(&slot_full[iv % SLOTS], (iv / SLOTS) & 1, abort_flag) &&
+                         (j >= nk || mbar_wait(&slot_full[ik % SLOTS], (ik / SLOTS) & 1, abort_flag)) &&
+                         mbar_wait(&p_full[t], (j - 1) & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t v_addr = kv_addr + (iv % SLOTS) * C::TILE_BYTES;
@@ -289,6 +293,14 @@ __global__ void __launch_bounds__(384, 1)
                     tmem_st32(o_addr + c * 32, r);
                 }
             }
+            // The two softmax warpgroups take turns for the exp2 pass (tile 0 of
+            // key tile j, then tile 1 of j, then tile 0 of j+1, ...), so each has
+            // the SFU to itself and the two tiles' MMAs interleave with it.
+            const bool my_turn_wait = (t == 0) ? (j > 0) : (j < nk0);
+            if (my_turn_wait) {
+                const bool wt = mbar_wait(&turn[t], (t == 0 ? j - 1 : j) & 1, abort_flag);
+                if (!__all_sync(0xffffffffu, wt)) { ok = false; break; }
+            }
             // pass 2: p = exp2(s * c2 - m), l += sum p, P (bf16) over the S columns.
             // Rows of a tile with no masked column (every warp of a non-diagonal,
             // non-tail tile) take a path with no per-element selects.
@@ -319,9 +331,13 @@ __global__ void __launch_bounds__(384, 1)
             }
             const float2 rs = fadd2(fadd2(rsum[0], rsum[1]), fadd2(rsum[2], rsum[3]));
             l += rs.x + rs.y;
+            // pass the turn on (tile 1 waits for tile 0 of this key tile only
+            // while tile 0 has one; tile 0 waits for tile 1 of the previous one)
+            if ((t == 0 || j + 1 < nk0) && lane == 0) mbar_arrive(&turn[1 - t]);
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&p_full[t]);
+            __syncwarp();  // every lane's P stores precede the warp's one arrival
+            if (lane == 0) mbar_arrive(&p_full[t]);
         }
         if (ok) {
             // PV(nk-2) is complete (S(nk-1) was seen), so the barrier is at most
