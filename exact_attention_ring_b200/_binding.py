@@ -140,9 +140,9 @@ def attn_selftest_bounded_wait(limit_us: int, stream=None):
 
 
 def decode_chunk(L: int, num_splits: int) -> int:
-    """Keys per split used by attn_decode_splitkv: 32 * ceil(ceil(L / S) / 32)."""
+    """Keys per split used by attn_decode_splitkv: 96 * ceil(ceil(L / S) / 96)."""
     per = -(-L // num_splits)
-    return -(-per // 32) * 32
+    return -(-per // 96) * 96
 
 
 # ------------------------------------------------------------- convenience --

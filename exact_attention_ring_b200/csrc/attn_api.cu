@@ -8,6 +8,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -63,9 +64,13 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     auto kern = attn_fwd_kernel<D, CAUSAL>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
-    const long long grid = static_cast<long long>(p.n_qblocks) * p.B * p.Hq;
-    if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-    kern<<<static_cast<unsigned>(grid), C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    // persistent grid: one CTA per SM, each walking its share of the work items
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        return ATTN_ERR_CUDA;
+    const int grid = p.n_items < sms ? p.n_items : sms;
+    kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -137,6 +142,9 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.lse = lse;
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N;
     p.n_qblocks = (N + 255) / 256;
+    const long long items = static_cast<long long>(p.n_qblocks) * B * Hq;
+    if (items > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    p.n_items = static_cast<int>(items);
     p.scale_log2 = scale * kLog2e;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d == 128) return causal ? launch_fwd<128, true>(tq, tk, tv, p, st) : launch_fwd<128, false>(tq, tk, tv, p, st);
@@ -154,9 +162,9 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, f
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (B > 65535 || num_splits > 0x7fffffff / 2) return ATTN_ERR_INVALID_ARG;
     const int per = (L + num_splits - 1) / num_splits;
-    const int chunk = (per + 31) / 32 * 32;
+    const int chunk = (per + 95) / 96 * 96;  // whole 96-key stages
     CUtensorMap tk, tv;
-    if (!make_map(&tk, k, d, L, B * Hkv, 32) || !make_map(&tv, v, d, L, B * Hkv, 32)) return ATTN_ERR_CUDA;
+    if (!make_map(&tk, k, d, L, B * Hkv, 96) || !make_map(&tv, v, d, L, B * Hkv, 96)) return ATTN_ERR_CUDA;
     DecodeParams p;
     p.q = static_cast<const __nv_bfloat16*>(q);
     p.o_part = o_part;
@@ -187,15 +195,31 @@ attn_status_t attn_combine(const float* o_part, const float* lse_part, void* o, 
 
 int attn_decode_default_splits(int B, int Hq, int Hkv, int L) {
     if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0) return 0;
-    constexpr int kSMs = 148, kWaves = 2, kMinKeys = 256;
+    // One decode block runs per SM (148 on B200) and streams its split at about
+    // the SM's share of HBM bandwidth after a fixed start-up worth ~260 keys.
+    // Pick the split count that maximises (busy fraction of the SM waves) x
+    // (streaming fraction chunk / (chunk + 260)).
+    constexpr int kSMs = 148, kStage = 96;
+    constexpr double kStartupKeys = 260.0;
     const int G = Hq / Hkv;
     const int gh = (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
     const long long units = static_cast<long long>(B) * Hkv * (G / gh);
-    long long s = (kSMs * kWaves + units - 1) / units;
-    const long long max_s = (L + kMinKeys - 1) / kMinKeys;
-    if (s > max_s) s = max_s;
-    if (s < 1) s = 1;
-    return static_cast<int>(s);
+    const int max_s = static_cast<int>(std::min<long long>((L + kStage - 1) / kStage, 4096));
+    int best_s = 1;
+    double best = -1.0;
+    for (int S = 1; S <= max_s; ++S) {
+        const long long per = (L + S - 1) / S;
+        const long long chunk = (per + kStage - 1) / kStage * kStage;
+        const long long nonempty = (L + chunk - 1) / chunk;
+        const long long waves = (units * S + kSMs - 1) / kSMs;
+        const double busy = static_cast<double>(units * nonempty) / static_cast<double>(kSMs * waves);
+        const double score = busy * (chunk / (chunk + kStartupKeys));
+        if (score > best + 1e-9) {
+            best = score;
+            best_s = S;
+        }
+    }
+    return best_s;
 }
 
 attn_status_t attn_device_status(attn_stream_t stream) {

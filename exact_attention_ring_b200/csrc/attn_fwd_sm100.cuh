@@ -6,30 +6,38 @@
 // value tiles stream past it; per row a running max m and denominator l are
 // kept, the accumulator is rescaled when the max moves, and O is divided by l
 // once at the end (FlashAttention V2 page: fewer non-matmul operations). Loop
-// order is the V2 one (query tiles outer, key/value tiles inner).
+// order is the V2 one (query tiles outer, key/value tiles inner), and work is
+// spread over thread blocks by sequence position as well as by head.
 //
-// B200 mapping. One CTA owns two 128-row query tiles of one head (256 rows)
-// that share every K/V tile; 384 threads, warp-specialised:
+// B200 mapping. A persistent grid (one CTA per SM) walks a list of work items;
+// an item is one 256-row query block of one (batch, head), processed as two
+// 128-row query tiles that share every K/V tile. Causal items are ordered
+// heaviest first and dealt to the CTAs in snake order. 384 threads,
+// warp-specialised:
 //   warps 0-3   softmax of query tile 0, one thread per row (TMEM lane);
 //   warps 4-7   softmax of query tile 1;
 //   warp 8, 9   MMA issuers, one per query tile. A thread that has just issued
 //               tcgen05.mma cannot act on an mbarrier for several hundred cycles,
 //               so two issuing warps keep the tensor core busy while each waits;
-//   warps 10,11 TMA producers: the two Q tiles, then K_j and V_j into a ring of
-//               shared-memory slots (full/empty mbarriers). One issuing thread
-//               streams TMA boxes one after another, so the boxes of every tile
-//               are split between two threads.
+//   warps 10,11 TMA producers: the Q tiles of each item, then K_j and V_j into a
+//               ring of shared-memory slots (full/empty mbarriers). One issuing
+//               thread streams TMA boxes one after another, so the boxes of
+//               every tile are split between two threads.
 // Per query tile t and key tile j:
 //   S_t = Q_t K_j^T           tcgen05.mma (A, B K-major in smem) -> TMEM S_t;
 //   softmax                   pass 1 reads S_t and takes the row max; when it has
 //                             grown by more than 2^8 (log2 units) O_t is rescaled
-//                             in TMEM (lazy rescale); pass 2 computes
+//                             in TMEM (lazy rescale); the two softmax warpgroups
+//                             then take turns for pass 2, which computes
 //                             p = exp2(s*scale*log2e - m) with one FMA, sums l in
 //                             fp32 and writes P_t as bf16 over the S_t columns;
 //   O_t += P_t V_j            tcgen05.mma with A = P_t from TMEM, B = V_j MN-major;
 // S_t(j+1) is issued after O_t += P_t(j) V_j by the same thread, so the tensor
 // pipe's issue order keeps P_t(j) intact until it has been read, and S_t(j+1)'s
-// completion implies that O_t holds every earlier P V product.
+// completion implies that O_t holds every earlier P V product. Between items
+// the next Q tile is loaded as soon as the last S MMA of its buffer completes,
+// and the next item's first P V waits only until the epilogue has read O_t.
+// Every barrier phase is counted across items.
 // TMEM columns: tile t uses S [256t, 256t+128) and O [256t+128, 256t+128+D).
 #pragma once
 
@@ -42,13 +50,14 @@ struct FwdParams {
     float* lse;        // [B, Hq, N]
     int B, Hq, Hkv, N;
     int n_qblocks;     // ceil(N / 256)
+    int n_items;       // n_qblocks * B * Hq
     float scale_log2;  // scale * log2(e)
 };
 
 template <int D>
 struct FwdCfg {
     static constexpr int BM = 128;                 // rows per query tile (= TMEM lanes)
-    static constexpr int TILES = 2;                // query tiles per CTA
+    static constexpr int TILES = 2;                // query tiles per work item
     static constexpr int BN = 128;                 // keys per K/V tile
     static constexpr int CHUNKS = D / 64;          // 64-element (128-byte) swizzle chunks per row
     static constexpr int Q_TILE_BYTES = BM * D * 2;
@@ -56,11 +65,42 @@ struct FwdCfg {
     static constexpr int SLOTS = (D == 128) ? 5 : 10;
     static constexpr int NUM_THREADS = 384;
     static constexpr int NUM_PRODUCERS = 2;
-    static constexpr int NUM_BARRIERS = 2 + 2 * SLOTS + 2 + 2 + 2 + 2 + 2;
+    // q_full, q_empty, slot_full, slot_empty, s_full, p_full, o_done, o_free, turn, drain
+    static constexpr int NUM_BARRIERS = 2 * 2 + 2 * SLOTS + 6 * 2;
     static constexpr int SMEM_BYTES = 1024 + TILES * Q_TILE_BYTES + SLOTS * TILE_BYTES + NUM_BARRIERS * 8 + 16;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: P <= 2^8 between rescales
 };
+
+// One work item: a 256-row query block of one (batch, head).
+struct FwdItem {
+    int qb, bh, b, h, hk;
+    int nk0, nk1;  // key tiles needed by query tile 0 and 1 (nk1 - nk0 is 0 or 1)
+};
+
+template <bool CAUSAL>
+__device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int w) {
+    FwdItem it;
+    const int bh_count = p.B * p.Hq;
+    const int rank = w / bh_count;
+    it.bh = w % bh_count;
+    it.qb = CAUSAL ? (p.n_qblocks - 1 - rank) : rank;  // heaviest causal blocks first
+    it.b = it.bh / p.Hq;
+    it.h = it.bh % p.Hq;
+    it.hk = it.h / (p.Hq / p.Hkv);
+    const int n_kv = (p.N + 127) / 128;
+    it.nk0 = CAUSAL ? min(2 * it.qb + 1, n_kv) : n_kv;
+    it.nk1 = CAUSAL ? min(2 * it.qb + 2, n_kv) : n_kv;
+    return it;
+}
+
+// The r-th work item of this CTA: rounds of gridDim.x items, dealt forwards in
+// even rounds and backwards in odd ones. Past the last item of this CTA every
+// later round is past the end too.
+__device__ __forceinline__ int fwd_work_index(int r) {
+    const int G = gridDim.x, c = blockIdx.x;
+    return r * G + ((r & 1) ? (G - 1 - c) : c);
+}
 
 // Max of 64 values with eight independent chains of 3-input max.
 __device__ __forceinline__ float max64(const float (&v)[64]) {
@@ -87,39 +127,31 @@ __global__ void __launch_bounds__(384, 1)
     uint8_t* sQ = smem;
     uint8_t* sKV = smem + C::TILES * C::Q_TILE_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + SLOTS * C::TILE_BYTES);
-    uint64_t* q_full = bars;                   // [2]
-    uint64_t* slot_full = q_full + 2;          // [SLOTS]
+    uint64_t* q_full = bars;                   // [2] Q tile t loaded
+    uint64_t* q_empty = q_full + 2;            // [2] last S of Q tile t's buffer done
+    uint64_t* slot_full = q_empty + 2;         // [SLOTS]
     uint64_t* slot_empty = slot_full + SLOTS;  // [SLOTS]
-    uint64_t* s_full = slot_empty + SLOTS;     // [2]
-    uint64_t* p_full = s_full + 2;             // [2]
-    uint64_t* o_done = p_full + 2;             // [2]
-    uint64_t* drain = o_done + 2;              // [2]
-    uint64_t* turn = drain + 2;                // [2] softmax ping-pong
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(turn + 2);
+    uint64_t* s_full = slot_empty + SLOTS;     // [2] S_t ready
+    uint64_t* p_full = s_full + 2;             // [2] P_t written (4 warp arrivals)
+    uint64_t* o_done = p_full + 2;             // [2] a P V product complete
+    uint64_t* o_free = o_done + 2;             // [2] epilogue has read O_t (4 warp arrivals)
+    uint64_t* turn = o_free + 2;               // [2] softmax ping-pong (4 warp arrivals)
+    uint64_t* drain = turn + 2;                // [2]
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // Work: one 256-row query block of one (batch, head); heaviest causal blocks first.
-    const int bh_count = p.B * p.Hq;
-    const int rank = blockIdx.x / bh_count;
-    const int bh = blockIdx.x % bh_count;
-    const int qb = CAUSAL ? (p.n_qblocks - 1 - rank) : rank;
-    const int b = bh / p.Hq, h = bh % p.Hq;
-    const int hk = h / (p.Hq / p.Hkv);
-    const int n_kv = (p.N + BN - 1) / BN;
-    // key tiles each query tile needs (tile 1 needs at most one more than tile 0)
-    const int nk0 = CAUSAL ? min(2 * qb + 1, n_kv) : n_kv;
-    const int nk1 = CAUSAL ? min(2 * qb + 2, n_kv) : n_kv;
-
     if (threadIdx.x == 0) {
         for (int t = 0; t < 2; ++t) {
             mbar_init(&q_full[t], C::CHUNKS);  // one expect_tx arrival per box
+            mbar_init(&q_empty[t], 1);
             mbar_init(&s_full[t], 1);
-            mbar_init(&p_full[t], 4);  // one arrival per softmax warp
+            mbar_init(&p_full[t], 4);
             mbar_init(&o_done[t], 1);
-            mbar_init(&drain[t], 1);
+            mbar_init(&o_free[t], 4);
             mbar_init(&turn[t], 4);
+            mbar_init(&drain[t], 1);
         }
         for (int i = 0; i < SLOTS; ++i) {
             mbar_init(&slot_full[i], C::CHUNKS);
@@ -139,48 +171,62 @@ __global__ void __launch_bounds__(384, 1)
 
     if (warp >= 10) {
         // ------------------------------------------------------ producers ---
-        // Box c of Q tile t, and box c of item i (K_j = item 2j, V_j = item
-        // 2j+1), go to producer (index * CHUNKS + c) % 2; each box arrives on its
-        // full barrier with its own byte count.
+        // Box c of Q tile t, and box c of K/V load g (K_j, V_j of an item are
+        // loads base + 2j, base + 2j + 1), go to producer (index * CHUNKS + c) % 2;
+        // each box arrives on its full barrier with its own byte count.
         if (lane == 0) {
             const int me = warp - 10;
-            const int zq = b * p.Hq + h, zkv = b * p.Hkv + hk;
             constexpr uint32_t BOX_BYTES = BN * 128;
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
+            bool ok = true;
+            int g = 0, it = 0;
+            for (int r = 0; ok; ++r, ++it) {
+                const int w = fwd_work_index(r);
+                if (w >= p.n_items) break;
+                const FwdItem item = fwd_item<CAUSAL>(p, w);
+                const int zq = item.b * p.Hq + item.h, zkv = item.b * p.Hkv + item.hk;
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
+                for (int t = 0; t < 2; ++t) {
+                    bool any = false;
 #pragma unroll
-                for (int c = 0; c < C::CHUNKS; ++c) {
-                    if ((t * C::CHUNKS + c) % C::NUM_PRODUCERS != me) continue;
-                    mbar_arrive_expect_tx(&q_full[t], BM * 128);
-                    tma_load_3d(sQ + t * C::Q_TILE_BYTES + c * BM * 128, &tm_q, &q_full[t], c * 64,
-                                qb * 2 * BM + t * BM, zq);
+                    for (int c = 0; c < C::CHUNKS; ++c) any |= ((t * C::CHUNKS + c) % C::NUM_PRODUCERS) == me;
+                    if (!any) continue;
+                    if (it > 0 && !mbar_wait(&q_empty[t], (it - 1) & 1, abort_flag)) { ok = false; break; }
+#pragma unroll
+                    for (int c = 0; c < C::CHUNKS; ++c) {
+                        if ((t * C::CHUNKS + c) % C::NUM_PRODUCERS != me) continue;
+                        mbar_arrive_expect_tx(&q_full[t], BM * 128);
+                        tma_load_3d(sQ + t * C::Q_TILE_BYTES + c * BM * 128, &tm_q, &q_full[t], c * 64,
+                                    item.qb * 2 * BM + t * BM, zq);
+                    }
                 }
-            int issued = 0;
-            for (int i = 0; i < 2 * nk1; ++i) {
-                bool mine = false;
+                for (int i = 0; ok && i < 2 * item.nk1; ++i) {
+                    const int gi = g + i;
+                    bool mine = false;
 #pragma unroll
-                for (int c = 0; c < C::CHUNKS; ++c) mine |= ((i * C::CHUNKS + c) % C::NUM_PRODUCERS) == me;
-                if (!mine) continue;
-                const int slot = i % SLOTS, use = i / SLOTS;
-                if (use > 0 && !mbar_wait(&slot_empty[slot], (use - 1) & 1, abort_flag)) break;
-                const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;
-                uint8_t* dst = sKV + slot * C::TILE_BYTES;
+                    for (int c = 0; c < C::CHUNKS; ++c) mine |= ((gi * C::CHUNKS + c) % C::NUM_PRODUCERS) == me;
+                    if (!mine) continue;
+                    const int slot = gi % SLOTS, use = gi / SLOTS;
+                    if (use > 0 && !mbar_wait(&slot_empty[slot], (use - 1) & 1, abort_flag)) { ok = false; break; }
+                    const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;
+                    uint8_t* dst = sKV + slot * C::TILE_BYTES;
 #pragma unroll
-                for (int c = 0; c < C::CHUNKS; ++c) {
-                    if ((i * C::CHUNKS + c) % C::NUM_PRODUCERS != me) continue;
-                    mbar_arrive_expect_tx(&slot_full[slot], BOX_BYTES);
-                    tma_load_3d(dst + c * BOX_BYTES, tm, &slot_full[slot], c * 64, (i >> 1) * BN, zkv);
+                    for (int c = 0; c < C::CHUNKS; ++c) {
+                        if ((gi * C::CHUNKS + c) % C::NUM_PRODUCERS != me) continue;
+                        mbar_arrive_expect_tx(&slot_full[slot], BOX_BYTES);
+                        tma_load_3d(dst + c * BOX_BYTES, tm, &slot_full[slot], c * 64, (i >> 1) * BN, zkv);
+                    }
                 }
-                issued = i + 1;
+                g += 2 * item.nk1;
             }
             // Let every copy in flight land before the CTA can exit.
-            mbar_wait(&q_full[0], 0, nullptr);
-            mbar_wait(&q_full[1], 0, nullptr);
-            for (int i = max(0, issued - SLOTS); i < issued; ++i)
-                mbar_wait(&slot_full[i % SLOTS], (i / SLOTS) & 1, nullptr);
+            if (it > 0) {
+                mbar_wait(&q_full[0], (it - 1) & 1, nullptr);
+                mbar_wait(&q_full[1], (it - 1) & 1, nullptr);
+            }
+            for (int i = max(0, g - SLOTS); i < g; ++i) mbar_wait(&slot_full[i % SLOTS], (i / SLOTS) & 1, nullptr);
         }
     } else if (warp >= 8) {
         // ---------------------------------------------------- MMA issuers ---
@@ -188,51 +234,63 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = make_idesc_bf16(BM, BN, 0, 0);
             constexpr uint32_t idesc_pv = make_idesc_bf16(BM, D, 0, 1);
-            const int nk = t ? nk1 : nk0;
             const uint32_t s_tmem = tmem + t * 256, o_tmem = s_tmem + 128;
             const uint32_t q_addr = smem_addr(sQ + t * C::Q_TILE_BYTES), kv_addr = smem_addr(sKV);
-            // item i (K_j = 2j, V_j = 2j+1) sits in slot i % SLOTS, use i / SLOTS
-            bool ok = mbar_wait(&q_full[t], 0, abort_flag) && mbar_wait(&slot_full[0], 0, abort_flag);
-            for (int j = 0; ok && j <= nk; ++j) {
-                if (j > 0) {
-                    // O_t += P_t(j-1) V_{j-1}; everything it and S_t(j) need is
-                    // awaited first so that both groups go out back to back.
-                    const int iv = 2 * j - 1, ik = 2 * j;
-                    // (the loads are usually long complete: check them first so
-                    // that only the wait for P sits on the critical path)
-                    ok = mbar_wait(&slot_full[iv % SLOTS], (iv / SLOTS) & 1, abort_flag) &&
-                         (j >= nk || mbar_wait(&slot_full[ik % SLOTS], (ik / SLOTS) & 1, abort_flag)) &&
-                         mbar_wait(&p_full[t], (j - 1) & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t v_addr = kv_addr + (iv % SLOTS) * C::TILE_BYTES;
+            bool ok = true;
+            int g = 0;        // K/V load index of the item's K_0
+            uint32_t np = 0;  // P_t handed over so far (p_full phases)
+            for (int r = 0, it = 0; ok; ++r, ++it) {
+                const int w = fwd_work_index(r);
+                if (w >= p.n_items) break;
+                const FwdItem item = fwd_item<CAUSAL>(p, w);
+                const int nk = t ? item.nk1 : item.nk0;
+                for (int j = 0; j <= nk; ++j) {
+                    const int ik = g + 2 * j, iv = g + 2 * j - 1;
+                    if (j == 0) {
+                        ok = mbar_wait(&q_full[t], it & 1, abort_flag) &&
+                             mbar_wait(&slot_full[ik % SLOTS], (ik / SLOTS) & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                    } else {
+                        // O_t += P_t(j-1) V_{j-1}. The loads (usually long done) are
+                        // checked before P so only the wait for P is on the critical
+                        // path; the first product of an item also needs the previous
+                        // item's epilogue to have read O_t.
+                        ok = mbar_wait(&slot_full[iv % SLOTS], (iv / SLOTS) & 1, abort_flag) &&
+                             (j >= nk || mbar_wait(&slot_full[ik % SLOTS], (ik / SLOTS) & 1, abort_flag)) &&
+                             (j > 1 || it == 0 || mbar_wait(&o_free[t], (it - 1) & 1, abort_flag)) &&
+                             mbar_wait(&p_full[t], np & 1, abort_flag);
+                        if (!ok) break;
+                        ++np;
+                        tc_fence_after();
+                        const uint32_t v_addr = kv_addr + (iv % SLOTS) * C::TILE_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk) {
-                        // V as the MN-major B operand: 16 keys = 2048 bytes per step;
-                        // LBO = distance between the 64-column chunks of the tile.
-                        const uint64_t bd = make_sdesc_sw128(v_addr + kk * 16 * 128, BN * 128, 1024);
-                        mma_ts(o_tmem, s_tmem + kk * 8, bd, idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < BN / 16; ++kk) {
+                            // V as the MN-major B operand: 16 keys = 2048 bytes per step;
+                            // LBO = distance between the 64-column chunks of the tile.
+                            const uint64_t bd = make_sdesc_sw128(v_addr + kk * 16 * 128, BN * 128, 1024);
+                            mma_ts(o_tmem, s_tmem + kk * 8, bd, idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
+                        }
+                        tc_commit(&o_done[t]);
+                        if (t == 1 && j - 1 >= item.nk0) mbar_arrive(&slot_empty[iv % SLOTS]);  // tile-1-only load
+                        tc_commit(&slot_empty[iv % SLOTS]);
+                        if (j >= nk) break;
                     }
-                    tc_commit(&o_done[t]);
-                    if (t == 1 && j - 1 >= nk0) mbar_arrive(&slot_empty[iv % SLOTS]);  // tile-1-only item
-                    tc_commit(&slot_empty[iv % SLOTS]);
-                    if (j >= nk) break;
-                } else {
-                    tc_fence_after();
-                }
-                // S_t(j) = Q_t K_j^T
-                const int ik = 2 * j;
-                const uint32_t k_addr = kv_addr + (ik % SLOTS) * C::TILE_BYTES;
+                    // S_t(j) = Q_t K_j^T
+                    const uint32_t k_addr = kv_addr + (ik % SLOTS) * C::TILE_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk & 3) * 32;  // 16 elements = 32 bytes inside the swizzle row
-                    const uint64_t ad = make_sdesc_sw128(q_addr + (kk >> 2) * (BM * 128) + koff, 16, 1024);
-                    const uint64_t bd = make_sdesc_sw128(k_addr + (kk >> 2) * (BN * 128) + koff, 16, 1024);
-                    mma_ss(s_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t koff = (kk & 3) * 32;  // 16 elements = 32 bytes inside the swizzle row
+                        const uint64_t ad = make_sdesc_sw128(q_addr + (kk >> 2) * (BM * 128) + koff, 16, 1024);
+                        const uint64_t bd = make_sdesc_sw128(k_addr + (kk >> 2) * (BN * 128) + koff, 16, 1024);
+                        mma_ss(s_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&s_full[t]);
+                    if (t == 1 && j >= item.nk0) mbar_arrive(&slot_empty[ik % SLOTS]);  // tile-1-only load
+                    tc_commit(&slot_empty[ik % SLOTS]);
+                    if (j == nk - 1) tc_commit(&q_empty[t]);  // Q_t buffer free once this S is done
                 }
-                tc_commit(&s_full[t]);
-                if (t == 1 && j >= nk0) mbar_arrive(&slot_empty[ik % SLOTS]);  // tile-1-only item
-                tc_commit(&slot_empty[ik % SLOTS]);
+                g += 2 * item.nk1;
             }
             // Every MMA must be complete before TMEM is released.
             tc_commit(&drain[t]);
@@ -244,127 +302,148 @@ __global__ void __launch_bounds__(384, 1)
         const int t = warp >> 2;
         const int quad = warp & 3;  // TMEM lane quadrant this warp may access
         const int row = quad * 32 + lane;
-        const int grow = qb * 2 * BM + t * BM + row;
-        const int q128 = 2 * qb + t;  // index of this query tile in 128-row units
-        const int nk = t ? nk1 : nk0;
         const uint32_t s_addr = tmem + t * 256 + (uint32_t(quad * 32) << 16);
         const uint32_t o_addr = s_addr + 128;
         const float c2 = p.scale_log2;
-        float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < nk; ++j) {
-            const bool w = mbar_wait(&s_full[t], j & 1, abort_flag);
-            if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-            tc_fence_after();
-            // valid key columns of this tile for this row: [0, lim)
-            int lim = BN;
-            if (CAUSAL && j == q128) lim = row + 1;
-            if (!CAUSAL && j * BN + BN > p.N) lim = p.N - j * BN;
-            // pass 1: row max
-            float mx = -INFINITY;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r[64];
-                tmem_ld64(s_addr + half * 64, r);
-                if (__any_sync(0xffffffffu, half * 64 + 64 > lim)) {
-#pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        if (half * 64 + i >= lim) r[i] = 0xff800000u;  // -inf
-                }
-                mx = fmaxf(mx, max64(reinterpret_cast<const float(&)[64]>(r)));
-            }
-            const float m_tile = mx * c2;
-            const bool need = m_tile > m_used + C::RESCALE_THRESHOLD;
-            float factor = 1.f;
-            if (need) {
-                factor = ex2_approx(m_used - m_tile);
-                m_used = m_tile;
-            }
-            l *= factor;
-            // S_t(j) completing implies O_t already holds every earlier P V
-            // product, so O_t can be rescaled now, before P_t(j) is released.
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(o_addr + c * 32, r);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * factor);
-                    tmem_st32(o_addr + c * 32, r);
-                }
-            }
-            // The two softmax warpgroups take turns for the exp2 pass (tile 0 of
-            // key tile j, then tile 1 of j, then tile 0 of j+1, ...), so each has
-            // the SFU to itself and the two tiles' MMAs interleave with it.
-            const bool my_turn_wait = (t == 0) ? (j > 0) : (j < nk0);
-            if (my_turn_wait) {
-                const bool wt = mbar_wait(&turn[t], (t == 0 ? j - 1 : j) & 1, abort_flag);
-                if (!__all_sync(0xffffffffu, wt)) { ok = false; break; }
-            }
-            // pass 2: p = exp2(s * c2 - m), l += sum p, P (bf16) over the S columns.
-            // Rows of a tile with no masked column (every warp of a non-diagonal,
-            // non-tail tile) take a path with no per-element selects.
-            const bool full = __all_sync(0xffffffffu, lim == BN);
-            const float2 c2x2 = make_float2(c2, c2), negm2 = make_float2(-m_used, -m_used);
-            float2 rsum[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) rsum[k] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r[64];
-                tmem_ld64(s_addr + half * 64, r);
-                if (!full) {
-#pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        if (half * 64 + i >= lim) r[i] = 0xff800000u;  // -inf: exp2 gives 0
-                }
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float2 y = ffma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
-                                           c2x2, negm2);
-                    const float2 pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
-                    rsum[i & 3] = fadd2(rsum[i & 3], pp);
-                    pk[i] = pack_bf16x2(pp.x, pp.y);
-                }
-                tmem_st32(s_addr + half * 32, pk);
-            }
-            const float2 rs = fadd2(fadd2(rsum[0], rsum[1]), fadd2(rsum[2], rsum[3]));
-            l += rs.x + rs.y;
-            // pass the turn on (tile 1 waits for tile 0 of this key tile only
-            // while tile 0 has one; tile 0 waits for tile 1 of the previous one)
-            if ((t == 0 || j + 1 < nk0) && lane == 0) mbar_arrive(&turn[1 - t]);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();  // every lane's P stores precede the warp's one arrival
-            if (lane == 0) mbar_arrive(&p_full[t]);
-        }
-        if (ok) {
-            // PV(nk-2) is complete (S(nk-1) was seen), so the barrier is at most
-            // one phase away and this parity wait is exact.
-            const bool w = mbar_wait(&o_done[t], (nk - 1) & 1, abort_flag);
-            if (__all_sync(0xffffffffu, w)) {
+        uint32_t ns = 0, nturn = 0, npv = 0;  // phases consumed so far, counted across items
+        for (int r = 0; ok; ++r) {
+            const int w = fwd_work_index(r);
+            if (w >= p.n_items) break;
+            const FwdItem item = fwd_item<CAUSAL>(p, w);
+            const bool has_next = fwd_work_index(r + 1) < p.n_items;
+            const int nk = t ? item.nk1 : item.nk0;
+            const int grow = item.qb * 2 * BM + t * BM + row;
+            const int q128 = 2 * item.qb + t;  // index of this query tile in 128-row units
+            float m_used = -INFINITY, l = 0.f;
+            for (int j = 0; j < nk; ++j) {
+                const bool w1 = mbar_wait(&s_full[t], ns & 1, abort_flag);
+                if (!__all_sync(0xffffffffu, w1)) { ok = false; break; }
+                ++ns;
                 tc_fence_after();
-                const float inv_l = 1.f / l;
-                __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + grow) * D;
+                // valid key columns of this tile for this row: [0, lim)
+                int lim = BN;
+                if (CAUSAL && j == q128) lim = row + 1;
+                if (!CAUSAL && j * BN + BN > p.N) lim = p.N - j * BN;
+                // pass 1: row max
+                float mx = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(o_addr + c * 32, r);
-                    uint32_t pk[16];
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t r2[64];
+                    tmem_ld64(s_addr + half * 64, r2);
+                    if (__any_sync(0xffffffffu, half * 64 + 64 > lim)) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
-                    if (grow < p.N) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+                        for (int i = 0; i < 64; ++i)
+                            if (half * 64 + i >= lim) r2[i] = 0xff800000u;  // -inf
+                    }
+                    mx = fmaxf(mx, max64(reinterpret_cast<const float(&)[64]>(r2)));
+                }
+                const float m_tile = mx * c2;
+                const bool need = m_tile > m_used + C::RESCALE_THRESHOLD;
+                float factor = 1.f;
+                if (need) {
+                    factor = ex2_approx(m_used - m_tile);
+                    m_used = m_tile;
+                }
+                l *= factor;
+                // S_t(j) completing implies O_t already holds every earlier P V
+                // product, so O_t can be rescaled now, before P_t(j) is released.
+                if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t r3[32];
+                        tmem_ld32(o_addr + c * 32, r3);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r3[i] = __float_as_uint(__uint_as_float(r3[i]) * factor);
+                        tmem_st32(o_addr + c * 32, r3);
                     }
                 }
-                if (grow < p.N)
-                    p.lse[static_cast<size_t>(bh) * p.N + grow] = (m_used + log2f(l)) * 0.69314718055994530942f;
+                // The two softmax warpgroups take turns for the exp2 pass: tile 0 of
+                // key tile j, then tile 1 of j, then tile 0 of j+1, ..., across items
+                // too (tile 1's extra causal key tile runs right after its previous
+                // one). Each then has the SFU to itself and the two tiles' MMAs
+                // interleave with it; strict alternation also keeps every turn
+                // barrier within one phase of its waiter.
+                const bool my_turn_wait = (t == 0) ? (r > 0 || j > 0) : (j < item.nk0);
+                if (my_turn_wait) {
+                    const bool wt = mbar_wait(&turn[t], nturn & 1, abort_flag);
+                    if (!__all_sync(0xffffffffu, wt)) { ok = false; break; }
+                    ++nturn;
+                }
+                // pass 2: p = exp2(s * c2 - m), l += sum p, P (bf16) over the S columns.
+                // Rows of a tile with no masked column (every warp of a non-diagonal,
+                // non-tail tile) take a path with no per-element selects.
+                const bool full = __all_sync(0xffffffffu, lim == BN);
+                const float2 c2x2 = make_float2(c2, c2), negm2 = make_float2(-m_used, -m_used);
+                float2 rsum[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) rsum[k] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t r2[64];
+                    tmem_ld64(s_addr + half * 64, r2);
+                    if (!full) {
+#pragma unroll
+                        for (int i = 0; i < 64; ++i)
+                            if (half * 64 + i >= lim) r2[i] = 0xff800000u;  // -inf: exp2 gives 0
+                    }
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float2 y = ffma2(make_float2(__uint_as_float(r2[2 * i]), __uint_as_float(r2[2 * i + 1])),
+                                               c2x2, negm2);
+                        const float2 pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+                        rsum[i & 3] = fadd2(rsum[i & 3], pp);
+                        pk[i] = pack_bf16x2(pp.x, pp.y);
+                    }
+                    tmem_st32(s_addr + half * 32, pk);
+                }
+                const float2 rs = fadd2(fadd2(rsum[0], rsum[1]), fadd2(rsum[2], rsum[3]));
+                l += rs.x + rs.y;
+                // pass the turn on: tile 0 always hands over to tile 1 of the same key
+                // tile; tile 1 hands back when tile 0 runs next (key tile j + 1 of
+                // this item, or key tile 0 of the next item)
+                const bool hand_over =
+                    (t == 0) || (j + 1 < item.nk0) || (j == item.nk1 - 1 && has_next);
+                if (hand_over && lane == 0) mbar_arrive(&turn[1 - t]);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();  // every lane's P stores precede the warp's one arrival
+                if (lane == 0) mbar_arrive(&p_full[t]);
             }
+            if (!ok) break;
+            // Epilogue. PV(nk-2) is complete (S(nk-1) was seen; for nk = 1 the
+            // previous item's epilogue waited for its last PV), so o_done is at
+            // most one phase away and this parity wait is exact.
+            npv += nk;
+            const bool w2 = mbar_wait(&o_done[t], (npv - 1) & 1, abort_flag);
+            if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
+            tc_fence_after();
+            const float inv_l = 1.f / l;
+            __nv_bfloat16* orow = p.o + (static_cast<size_t>(item.bh) * p.N + grow) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r3[32];
+                tmem_ld32(o_addr + c * 32, r3);
+                if (c == D / 32 - 1) {
+                    // O_t is in registers: the next item's first P V may overwrite it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&o_free[t]);
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(__uint_as_float(r3[2 * i]) * inv_l, __uint_as_float(r3[2 * i + 1]) * inv_l);
+                if (grow < p.N) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                }
+            }
+            if (grow < p.N)
+                p.lse[static_cast<size_t>(item.bh) * p.N + grow] = (m_used + log2f(l)) * 0.69314718055994530942f;
         }
     }
 

@@ -116,19 +116,22 @@ def test_default_splits(lib):
     f = lib.attn_decode_default_splits
     f.restype = ctypes.c_int
     assert f(0, 32, 8, 100) == 0 and f(1, 30, 8, 100) == 0
-    # B=1, 8 KV heads, 4 query heads each: 8 blocks per split; about 2 x 148 blocks wanted
-    assert f(1, 32, 8, 32768) == 37
-    assert f(1, 32, 8, 4096) == 16        # capped by >= 256 keys per split
-    assert f(8, 32, 8, 131072) == 5
+    # B=1, 8 KV heads, 4 query heads each: 8 blocks per split -> one wave of 144
+    assert f(1, 32, 8, 32768) == 18
+    assert f(1, 32, 8, 131072) == 18
+    # B=8: 64 blocks per split; 9 splits = 576 blocks = 3.9 waves of 148
+    assert f(8, 32, 8, 32768) == 9
+    assert f(8, 32, 8, 131072) == 16
     assert f(1, 1, 1, 1) == 1
     for L in (1, 31, 257, 100000):
         s = f(2, 16, 4, L)
-        assert 1 <= s <= L
+        assert 1 <= s <= -(-L // 96)
 
 
 def test_decode_chunk_rule():
     from exact_attention_ring_b200 import decode_chunk
-    assert decode_chunk(4096, 16) == 256
-    assert decode_chunk(32768, 37) == 896
-    assert decode_chunk(100, 64) == 32
-    assert decode_chunk(1, 1) == 32
+    assert decode_chunk(4096, 16) == 288
+    assert decode_chunk(32768, 37) == 960
+    assert decode_chunk(100, 64) == 96
+    assert decode_chunk(1, 1) == 96
+    assert decode_chunk(131072, 5) == 26304
