@@ -50,7 +50,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic per launch from one ncu capture, valid only for the kernel source
 # it was taken on (sha256 of the kernel file, first 16 hex digits).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # decode_splitkv_kernel<128,4>, B1 Hq32 Hkv8 L131072 d128 (the bench's decode workload)
+    "decode": {"bytes_per_launch": 536985088 + 4048128, "source_sha": "67c9877f6eecc387"},
+}
 
 
 def kernel_sha(name: str) -> str:
