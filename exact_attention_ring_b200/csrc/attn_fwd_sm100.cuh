@@ -14,8 +14,10 @@
 // 128-row query tiles that share every K/V tile. Causal items are ordered
 // heaviest first and dealt to the CTAs in snake order. 384 threads,
 // warp-specialised:
-//   warps 0-3   softmax of query tile 0, one thread per row (TMEM lane);
-//   warps 4-7   softmax of query tile 1;
+//   warps 0-3   softmax of query tile 0, one thread per row (TMEM lane), and
+//               its epilogue: O/l to bf16, staged per warp in shared memory
+//               (32 rows x 32 columns at a time) and written by TMA stores;
+//   warps 4-7   the same for query tile 1;
 //   warp 8, 9   MMA issuers, one per query tile. A thread that has just issued
 //               tcgen05.mma cannot act on an mbarrier for several hundred cycles,
 //               so two issuing warps keep the tensor core busy while each waits;
@@ -62,12 +64,14 @@ struct FwdCfg {
     static constexpr int CHUNKS = D / 64;          // 64-element (128-byte) swizzle chunks per row
     static constexpr int Q_TILE_BYTES = BM * D * 2;
     static constexpr int TILE_BYTES = BN * D * 2;  // one K or V tile
-    static constexpr int SLOTS = (D == 128) ? 5 : 10;
+    static constexpr int SLOTS = (D == 128) ? 4 : 10;
+    static constexpr int STAGE_O_BYTES = 32 * 32 * 2;  // per softmax warp: 32 rows x 32 bf16
     static constexpr int NUM_THREADS = 384;
     static constexpr int NUM_PRODUCERS = 2;
     // q_full, q_empty, slot_full, slot_empty, s_full, p_full, o_done, o_free, turn, drain
     static constexpr int NUM_BARRIERS = 2 * 2 + 2 * SLOTS + 6 * 2;
-    static constexpr int SMEM_BYTES = 1024 + TILES * Q_TILE_BYTES + SLOTS * TILE_BYTES + NUM_BARRIERS * 8 + 16;
+    static constexpr int SMEM_BYTES =
+        1024 + TILES * Q_TILE_BYTES + SLOTS * TILE_BYTES + 8 * STAGE_O_BYTES + NUM_BARRIERS * 8 + 16;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: P <= 2^8 between rescales
 };
@@ -119,14 +123,16 @@ __device__ __forceinline__ float max64(const float (&v)[64]) {
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                    const FwdParams p) {
     using C = FwdCfg<D>;
     constexpr int BM = C::BM, BN = C::BN, SLOTS = C::SLOTS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
     uint8_t* sKV = smem + C::TILES * C::Q_TILE_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + SLOTS * C::TILE_BYTES);
+    uint8_t* sO = sKV + SLOTS * C::TILE_BYTES;  // [8 warps][32 rows][32 bf16] epilogue staging
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sO + 8 * C::STAGE_O_BYTES);
     uint64_t* q_full = bars;                   // [2] Q tile t loaded
     uint64_t* q_empty = q_full + 2;            // [2] last S of Q tile t's buffer done
     uint64_t* slot_full = q_empty + 2;         // [SLOTS]
@@ -420,7 +426,8 @@ __global__ void __launch_bounds__(384, 1)
             if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
             tc_fence_after();
             const float inv_l = 1.f / l;
-            __nv_bfloat16* orow = p.o + (static_cast<size_t>(item.bh) * p.N + grow) * D;
+            uint8_t* stage = sO + warp * C::STAGE_O_BYTES;
+            const int row0 = item.qb * 2 * BM + t * BM + quad * 32;  // first row of this warp
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t r3[32];
@@ -435,11 +442,17 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     pk[i] = pack_bf16x2(__uint_as_float(r3[2 * i]) * inv_l, __uint_as_float(r3[2 * i + 1]) * inv_l);
-                if (grow < p.N) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+                // the staging buffer must have been read by this warp's previous store
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+                uint4* dst = reinterpret_cast<uint4*>(stage + lane * 64);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && row0 < p.N) {  // rows >= N inside the box are clipped
+                    tma_store_3d(&tm_o, stage, c * 32, row0, item.bh);
+                    bulk_commit_group();
                 }
             }
             if (grow < p.N)
@@ -447,6 +460,7 @@ __global__ void __launch_bounds__(384, 1)
         }
     }
 
+    if (warp < 8 && lane == 0) bulk_wait_group_read0();  // staged O read out before exit
     tc_fence_before();
     __syncthreads();
     if (warp == 8) {
