@@ -37,20 +37,18 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// bf16 tensor viewed as [planes, rows, D] with a {box_cols, box_rows, 1} box;
-// loads use box_cols = 64 with 128-byte swizzle (rows past `rows` read as
-// zero), stores use a plain box (rows past `rows` are clipped).
-bool make_map(CUtensorMap* map, const void* base, int D, int rows, int planes, int box_rows, int box_cols = 64,
-              bool swizzle = true) {
+// bf16 tensor viewed as [planes, rows, D] with a {64, box_rows, 1} box and
+// 128-byte swizzle; rows past `rows` read as zero.
+bool make_map(CUtensorMap* map, const void* base, int D, int rows, int planes, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(rows), cuuint64_t(planes)};
     const cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(D) * 2 * cuuint64_t(rows)};
-    const cuuint32_t box[3] = {cuuint32_t(box_cols), cuuint32_t(box_rows), 1};
+    const cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool aligned16(const void* ptr) { return ptr != nullptr && (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
@@ -60,8 +58,8 @@ bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D, bool CAUSAL>
-attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
-                         const FwdParams& p, cudaStream_t stream) {
+attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                         cudaStream_t stream) {
     using C = FwdCfg<D>;
     auto kern = attn_fwd_kernel<D, CAUSAL>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
@@ -72,7 +70,7 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
         return ATTN_ERR_CUDA;
     const int grid = p.n_items < sms ? p.n_items : sms;
-    kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
+    kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -135,9 +133,9 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
         return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (static_cast<long long>(B) * Hq > 65535LL * 1024) return ATTN_ERR_INVALID_ARG;
-    CUtensorMap tq, tk, tv, to;
+    CUtensorMap tq, tk, tv;
     if (!make_map(&tq, q, d, N, B * Hq, 128) || !make_map(&tk, k, d, N, B * Hkv, 128) ||
-        !make_map(&tv, v, d, N, B * Hkv, 128) || !make_map(&to, o, d, N, B * Hq, 32, 32, false))
+        !make_map(&tv, v, d, N, B * Hkv, 128))
         return ATTN_ERR_CUDA;
     FwdParams p;
     p.o = static_cast<__nv_bfloat16*>(o);
@@ -149,9 +147,8 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.n_items = static_cast<int>(items);
     p.scale_log2 = scale * kLog2e;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (d == 128)
-        return causal ? launch_fwd<128, true>(tq, tk, tv, to, p, st) : launch_fwd<128, false>(tq, tk, tv, to, p, st);
-    return causal ? launch_fwd<64, true>(tq, tk, tv, to, p, st) : launch_fwd<64, false>(tq, tk, tv, to, p, st);
+    if (d == 128) return causal ? launch_fwd<128, true>(tq, tk, tv, p, st) : launch_fwd<128, false>(tq, tk, tv, p, st);
+    return causal ? launch_fwd<64, true>(tq, tk, tv, p, st) : launch_fwd<64, false>(tq, tk, tv, p, st);
 }
 
 attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, float* o_part, float* lse_part,

@@ -16,7 +16,9 @@
 // warp-specialised:
 //   warps 0-3   softmax of query tile 0, one thread per row (TMEM lane), and
 //               its epilogue: O/l to bf16, staged per warp in shared memory
-//               (32 rows x 32 columns at a time) and written by TMA stores;
+//               (32 rows x 64 columns at a time, 16-byte chunks XOR-swizzled)
+//               and read back so that every store writes whole 128-byte row
+//               segments;
 //   warps 4-7   the same for query tile 1;
 //   warp 8, 9   MMA issuers, one per query tile. A thread that has just issued
 //               tcgen05.mma cannot act on an mbarrier for several hundred cycles,
@@ -65,7 +67,7 @@ struct FwdCfg {
     static constexpr int Q_TILE_BYTES = BM * D * 2;
     static constexpr int TILE_BYTES = BN * D * 2;  // one K or V tile
     static constexpr int SLOTS = (D == 128) ? 4 : 10;
-    static constexpr int STAGE_O_BYTES = 32 * 32 * 2;  // per softmax warp: 32 rows x 32 bf16
+    static constexpr int STAGE_O_BYTES = 32 * 64 * 2;  // per softmax warp: 32 rows x 64 bf16
     static constexpr int NUM_THREADS = 384;
     static constexpr int NUM_PRODUCERS = 2;
     // q_full, q_empty, slot_full, slot_empty, s_full, p_full, o_done, o_free, turn, drain
@@ -123,15 +125,14 @@ __device__ __forceinline__ float max64(const float (&v)[64]) {
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                    const FwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
     using C = FwdCfg<D>;
     constexpr int BM = C::BM, BN = C::BN, SLOTS = C::SLOTS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
     uint8_t* sKV = smem + C::TILES * C::Q_TILE_BYTES;
-    uint8_t* sO = sKV + SLOTS * C::TILE_BYTES;  // [8 warps][32 rows][32 bf16] epilogue staging
+    uint8_t* sO = sKV + SLOTS * C::TILE_BYTES;  // [8 warps][32 rows][64 bf16] epilogue staging
     uint64_t* bars = reinterpret_cast<uint64_t*>(sO + 8 * C::STAGE_O_BYTES);
     uint64_t* q_full = bars;                   // [2] Q tile t loaded
     uint64_t* q_empty = q_full + 2;            // [2] last S of Q tile t's buffer done
@@ -193,29 +194,15 @@ __global__ void __launch_bounds__(384, 1)
                 if (w >= p.n_items) break;
                 const FwdItem item = fwd_item<CAUSAL>(p, w);
                 const int zq = item.b * p.Hq + item.h, zkv = item.b * p.Hkv + item.hk;
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    bool any = false;
-#pragma unroll
-                    for (int c = 0; c < C::CHUNKS; ++c) any |= ((t * C::CHUNKS + c) % C::NUM_PRODUCERS) == me;
-                    if (!any) continue;
-                    if (it > 0 && !mbar_wait(&q_empty[t], (it - 1) & 1, abort_flag)) { ok = false; break; }
-#pragma unroll
-                    for (int c = 0; c < C::CHUNKS; ++c) {
-                        if ((t * C::CHUNKS + c) % C::NUM_PRODUCERS != me) continue;
-                        mbar_arrive_expect_tx(&q_full[t], BM * 128);
-                        tma_load_3d(sQ + t * C::Q_TILE_BYTES + c * BM * 128, &tm_q, &q_full[t], c * 64,
-                                    item.qb * 2 * BM + t * BM, zq);
-                    }
-                }
-                for (int i = 0; ok && i < 2 * item.nk1; ++i) {
+                // issue (this producer's boxes of) K/V load i of the item
+                auto issue_kv = [&](int i) -> bool {
                     const int gi = g + i;
                     bool mine = false;
 #pragma unroll
                     for (int c = 0; c < C::CHUNKS; ++c) mine |= ((gi * C::CHUNKS + c) % C::NUM_PRODUCERS) == me;
-                    if (!mine) continue;
+                    if (!mine) return true;
                     const int slot = gi % SLOTS, use = gi / SLOTS;
-                    if (use > 0 && !mbar_wait(&slot_empty[slot], (use - 1) & 1, abort_flag)) { ok = false; break; }
+                    if (use > 0 && !mbar_wait(&slot_empty[slot], (use - 1) & 1, abort_flag)) return false;
                     const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;
                     uint8_t* dst = sKV + slot * C::TILE_BYTES;
 #pragma unroll
@@ -224,7 +211,30 @@ __global__ void __launch_bounds__(384, 1)
                         mbar_arrive_expect_tx(&slot_full[slot], BOX_BYTES);
                         tma_load_3d(dst + c * BOX_BYTES, tm, &slot_full[slot], c * 64, (i >> 1) * BN, zkv);
                     }
-                }
+                    return true;
+                };
+                // issue (this producer's boxes of) Q tile t of the item
+                auto issue_q = [&](int t) -> bool {
+                    bool any = false;
+#pragma unroll
+                    for (int c = 0; c < C::CHUNKS; ++c) any |= ((t * C::CHUNKS + c) % C::NUM_PRODUCERS) == me;
+                    if (!any) return true;
+                    if (it > 0 && !mbar_wait(&q_empty[t], (it - 1) & 1, abort_flag)) return false;
+#pragma unroll
+                    for (int c = 0; c < C::CHUNKS; ++c) {
+                        if ((t * C::CHUNKS + c) % C::NUM_PRODUCERS != me) continue;
+                        mbar_arrive_expect_tx(&q_full[t], BM * 128);
+                        tma_load_3d(sQ + t * C::Q_TILE_BYTES + c * BM * 128, &tm_q, &q_full[t], c * 64,
+                                    item.qb * 2 * BM + t * BM, zq);
+                    }
+                    return true;
+                };
+                // Order: Q tile 0 (its buffer frees at tile 0's last S of the previous
+                // item), K_0 and V_0 (slots the previous item's last tiles release),
+                // then Q tile 1 (free after tile 1's last S, one key tile later in a
+                // causal item), then the rest.
+                ok = issue_q(0) && issue_kv(0) && issue_kv(1) && issue_q(1);
+                for (int i = 2; ok && i < 2 * item.nk1; ++i) ok = issue_kv(i);
                 g += 2 * item.nk1;
             }
             // Let every copy in flight land before the CTA can exit.
@@ -429,38 +439,48 @@ __global__ void __launch_bounds__(384, 1)
             uint8_t* stage = sO + warp * C::STAGE_O_BYTES;
             const int row0 = item.qb * 2 * BM + t * BM + quad * 32;  // first row of this warp
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r3[32];
-                tmem_ld32(o_addr + c * 32, r3);
-                if (c == D / 32 - 1) {
-                    // O_t is in registers: the next item's first P V may overwrite it
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&o_free[t]);
-                }
-                uint32_t pk[16];
+            for (int half = 0; half < D / 64; ++half) {
+                // this lane's row, columns [64*half, 64*half + 64): 128 bytes as 8
+                // chunks of 16; chunk i of row r sits at slot i ^ (r & 7)
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    pk[i] = pack_bf16x2(__uint_as_float(r3[2 * i]) * inv_l, __uint_as_float(r3[2 * i + 1]) * inv_l);
-                // the staging buffer must have been read by this warp's previous store
-                if (lane == 0) bulk_wait_group_read0();
-                __syncwarp();
-                uint4* dst = reinterpret_cast<uint4*>(stage + lane * 64);
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    const int c = half * 2 + c2;
+                    uint32_t r3[32];
+                    tmem_ld32(o_addr + c * 32, r3);
+                    if (c == D / 32 - 1) {
+                        // O_t is in registers: the next item's first P V may overwrite it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&o_free[t]);
+                    }
 #pragma unroll
-                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0 && row0 < p.N) {  // rows >= N inside the box are clipped
-                    tma_store_3d(&tm_o, stage, c * 32, row0, item.bh);
-                    bulk_commit_group();
+                    for (int i = 0; i < 4; ++i) {
+                        const int chunk = c2 * 4 + i;
+                        const uint4 v4 = make_uint4(
+                            pack_bf16x2(__uint_as_float(r3[8 * i + 0]) * inv_l, __uint_as_float(r3[8 * i + 1]) * inv_l),
+                            pack_bf16x2(__uint_as_float(r3[8 * i + 2]) * inv_l, __uint_as_float(r3[8 * i + 3]) * inv_l),
+                            pack_bf16x2(__uint_as_float(r3[8 * i + 4]) * inv_l, __uint_as_float(r3[8 * i + 5]) * inv_l),
+                            pack_bf16x2(__uint_as_float(r3[8 * i + 6]) * inv_l, __uint_as_float(r3[8 * i + 7]) * inv_l));
+                        *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = v4;
+                    }
                 }
+                __syncwarp();
+                // read back: lane = 8 * (row within a group of 4) + chunk, 4 rows per store
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int rr = 4 * k + (lane >> 3), chunk = lane & 7;
+                    const uint4 v4 = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((chunk ^ (rr & 7)) << 4));
+                    if (row0 + rr < p.N)
+                        *reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(item.bh) * p.N + row0 + rr) * D +
+                                                  half * 64 + chunk * 8) = v4;
+                }
+                __syncwarp();
             }
             if (grow < p.N)
                 p.lse[static_cast<size_t>(item.bh) * p.N + grow] = (m_used + log2f(l)) * 0.69314718055994530942f;
         }
     }
 
-    if (warp < 8 && lane == 0) bulk_wait_group_read0();  // staged O read out before exit
     tc_fence_before();
     __syncthreads();
     if (warp == 8) {
