@@ -34,8 +34,12 @@
 //                             in TMEM (lazy rescale); the two softmax warpgroups
 //                             then take turns for pass 2, which computes
 //                             p = exp2(s*scale*log2e - m) with one FMA, sums l in
-//                             fp32 and writes P_t as bf16 over the S_t columns;
-//   O_t += P_t V_j            tcgen05.mma with A = P_t from TMEM, B = V_j MN-major;
+//                             fp32 and writes P_t as bf16 over the S_t columns,
+//                             announcing each half (64 keys) as it lands;
+//   O_t += P_t V_j            tcgen05.mma with A = P_t from TMEM, B = V_j MN-major,
+//                             the first 64 keys while the softmax still works on
+//                             the second 64. The issuer waits on P by polling
+//                             (a suspended wait resumes late).
 // S_t(j+1) is issued after O_t += P_t(j) V_j by the same thread, so the tensor
 // pipe's issue order keeps P_t(j) intact until it has been read, and S_t(j+1)'s
 // completion implies that O_t holds every earlier P V product. Between items
@@ -70,8 +74,8 @@ struct FwdCfg {
     static constexpr int STAGE_O_BYTES = 32 * 64 * 2;  // per softmax warp: 32 rows x 64 bf16
     static constexpr int NUM_THREADS = 384;
     static constexpr int NUM_PRODUCERS = 2;
-    // q_full, q_empty, slot_full, slot_empty, s_full, p_full, o_done, o_free, turn, drain
-    static constexpr int NUM_BARRIERS = 2 * 2 + 2 * SLOTS + 6 * 2;
+    // q_full, q_empty, slot_full, slot_empty, s_full, p_full, o_done, o_free, turn, drain, p_half
+    static constexpr int NUM_BARRIERS = 2 * 2 + 2 * SLOTS + 7 * 2;
     static constexpr int SMEM_BYTES =
         1024 + TILES * Q_TILE_BYTES + SLOTS * TILE_BYTES + 8 * STAGE_O_BYTES + NUM_BARRIERS * 8 + 16;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -144,7 +148,8 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* o_free = o_done + 2;             // [2] epilogue has read O_t (4 warp arrivals)
     uint64_t* turn = o_free + 2;               // [2] softmax ping-pong (4 warp arrivals)
     uint64_t* drain = turn + 2;                // [2]
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
+    uint64_t* p_half = drain + 2;              // [2] first half of P_t written (4 warp arrivals)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(p_half + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -159,6 +164,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&o_free[t], 4);
             mbar_init(&turn[t], 4);
             mbar_init(&drain[t], 1);
+            mbar_init(&p_half[t], 4);
         }
         for (int i = 0; i < SLOTS; ++i) {
             mbar_init(&slot_full[i], C::CHUNKS);
@@ -275,18 +281,24 @@ __global__ void __launch_bounds__(384, 1)
                         ok = mbar_wait(&slot_full[iv % SLOTS], (iv / SLOTS) & 1, abort_flag) &&
                              (j >= nk || mbar_wait(&slot_full[ik % SLOTS], (ik / SLOTS) & 1, abort_flag)) &&
                              (j > 1 || it == 0 || mbar_wait(&o_free[t], (it - 1) & 1, abort_flag)) &&
-                             mbar_wait(&p_full[t], np & 1, abort_flag);
+                             mbar_wait_spin(&p_half[t], np & 1, abort_flag);
                         if (!ok) break;
-                        ++np;
                         tc_fence_after();
                         const uint32_t v_addr = kv_addr + (iv % SLOTS) * C::TILE_BYTES;
 #pragma unroll
                         for (int kk = 0; kk < BN / 16; ++kk) {
+                            if (kk == BN / 32) {
+                                ok = mbar_wait_spin(&p_full[t], np & 1, abort_flag);
+                                if (!ok) break;
+                                tc_fence_after();
+                            }
                             // V as the MN-major B operand: 16 keys = 2048 bytes per step;
                             // LBO = distance between the 64-column chunks of the tile.
                             const uint64_t bd = make_sdesc_sw128(v_addr + kk * 16 * 128, BN * 128, 1024);
                             mma_ts(o_tmem, s_tmem + kk * 8, bd, idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
                         }
+                        if (!ok) break;
+                        ++np;
                         tc_commit(&o_done[t]);
                         if (t == 1 && j - 1 >= item.nk0) mbar_arrive(&slot_empty[iv % SLOTS]);  // tile-1-only load
                         tc_commit(&slot_empty[iv % SLOTS]);
@@ -376,10 +388,11 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 // The two softmax warpgroups take turns for the exp2 pass: tile 0 of
                 // key tile j, then tile 1 of j, then tile 0 of j+1, ..., across items
-                // too (tile 1's extra causal key tile runs right after its previous
-                // one). Each then has the SFU to itself and the two tiles' MMAs
+                // too. Each then has the SFU to itself and the two tiles' MMAs
                 // interleave with it; strict alternation also keeps every turn
-                // barrier within one phase of its waiter.
+                // barrier within one phase of its waiter. Tile 1's extra causal key
+                // tile (the diagonal one of its rows) takes no turn: it overlaps
+                // tile 0's first key tile of the next item.
                 const bool my_turn_wait = (t == 0) ? (r > 0 || j > 0) : (j < item.nk0);
                 if (my_turn_wait) {
                     const bool wt = mbar_wait(&turn[t], nturn & 1, abort_flag);
@@ -413,14 +426,21 @@ __global__ void __launch_bounds__(384, 1)
                         pk[i] = pack_bf16x2(pp.x, pp.y);
                     }
                     tmem_st32(s_addr + half * 32, pk);
+                    if (half == 0) {
+                        // keys 0-63 of P_t are in TMEM: their P V steps may start
+                        tmem_st_wait();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&p_half[t]);
+                    }
                 }
                 const float2 rs = fadd2(fadd2(rsum[0], rsum[1]), fadd2(rsum[2], rsum[3]));
                 l += rs.x + rs.y;
                 // pass the turn on: tile 0 always hands over to tile 1 of the same key
-                // tile; tile 1 hands back when tile 0 runs next (key tile j + 1 of
-                // this item, or key tile 0 of the next item)
+                // tile; tile 1 hands back after each key tile it shares with tile 0
+                // (for key tile j + 1 of this item, or key tile 0 of the next item)
                 const bool hand_over =
-                    (t == 0) || (j + 1 < item.nk0) || (j == item.nk1 - 1 && has_next);
+                    (t == 0) || (j + 1 < item.nk0) || (j == item.nk0 - 1 && has_next);
                 if (hand_over && lane == 0) mbar_arrive(&turn[1 - t]);
                 tmem_st_wait();
                 tc_fence_before();

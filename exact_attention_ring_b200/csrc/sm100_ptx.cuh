@@ -98,6 +98,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     return mbar_wait_slow(bar, parity, abort, limit_ns);
 }
 
+// Waits by non-blocking probes only (no suspended try_wait), for the waits on
+// the critical path of a waiter that has nothing else to do.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               uint64_t limit_ns = kWaitLimitNs) {
+#pragma unroll 1
+    for (int i = 0; i < 8192; ++i)
+        if (mbar_test_wait(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, abort, limit_ns);
+}
+
 // --------------------------------------------------------- TMA / bulk ----
 __device__ __forceinline__ void tma_prefetch_desc(const void* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
