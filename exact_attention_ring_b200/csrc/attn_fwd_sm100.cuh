@@ -299,10 +299,12 @@ __global__ void __launch_bounds__(384, 1)
                         }
                         if (!ok) break;
                         ++np;
-                        tc_commit(&o_done[t]);
-                        if (t == 1 && j - 1 >= item.nk0) mbar_arrive(&slot_empty[iv % SLOTS]);  // tile-1-only load
-                        tc_commit(&slot_empty[iv % SLOTS]);
-                        if (j >= nk) break;
+                        if (j >= nk) {
+                            tc_commit(&o_done[t]);
+                            if (t == 1 && j - 1 >= item.nk0) mbar_arrive(&slot_empty[iv % SLOTS]);  // tile-1-only load
+                            tc_commit(&slot_empty[iv % SLOTS]);
+                            break;
+                        }
                     }
                     // S_t(j) = Q_t K_j^T
                     const uint32_t k_addr = kv_addr + (ik % SLOTS) * C::TILE_BYTES;
@@ -314,6 +316,13 @@ __global__ void __launch_bounds__(384, 1)
                         mma_ss(s_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
                     }
                     tc_commit(&s_full[t]);
+                    // P V(j-1) is signalled after S(j) so that the softmax hears of
+                    // S first; each commit covers every earlier MMA of this thread.
+                    if (j > 0) {
+                        tc_commit(&o_done[t]);
+                        if (t == 1 && j - 1 >= item.nk0) mbar_arrive(&slot_empty[iv % SLOTS]);  // tile-1-only load
+                        tc_commit(&slot_empty[iv % SLOTS]);
+                    }
                     if (t == 1 && j >= item.nk0) mbar_arrive(&slot_empty[ik % SLOTS]);  // tile-1-only load
                     tc_commit(&slot_empty[ik % SLOTS]);
                     if (j == nk - 1) tc_commit(&q_empty[t]);  // Q_t buffer free once this S is done
