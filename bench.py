@@ -53,6 +53,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     # decode_splitkv_kernel<128,4>, B1 Hq32 Hkv8 L131072 d128 (the bench's decode workload)
     "decode": {"bytes_per_launch": 536985088 + 4048128, "source_sha": "67c9877f6eecc387"},
+    # attn_fwd_kernel<128,causal / non-causal>, B2 H32 N2048 d128 (the bench's prefill workloads),
+    # read + write with cold caches (ncu flushes them before each captured launch)
+    "attn_fwd_causal": {"bytes_per_launch": 140439296 + 16052992, "source_sha": "b49431b3b24c0650"},
+    "attn_fwd_noncausal": {"bytes_per_launch": 239008256 + 26497792, "source_sha": "b49431b3b24c0650"},
 }
 
 
