@@ -55,8 +55,8 @@ NCU_TRAFFIC = {
     "decode": {"bytes_per_launch": 536985088 + 4048128, "source_sha": "67c9877f6eecc387"},
     # attn_fwd_kernel<128,causal / non-causal>, B2 H32 N2048 d128 (the bench's prefill workloads),
     # read + write with cold caches (ncu flushes them before each captured launch)
-    "attn_fwd_causal": {"bytes_per_launch": 140439296 + 16052992, "source_sha": "b49431b3b24c0650"},
-    "attn_fwd_noncausal": {"bytes_per_launch": 239008256 + 26497792, "source_sha": "b49431b3b24c0650"},
+    "attn_fwd_causal": {"bytes_per_launch": 148234496 + 16394240, "source_sha": "ed115c8fd1b2acdf"},
+    "attn_fwd_noncausal": {"bytes_per_launch": 259220992 + 27508224, "source_sha": "ed115c8fd1b2acdf"},
 }
 
 

@@ -8,8 +8,14 @@ the library has not been built, importing this package raises.
 Low-level calls (same names and arguments as the C ABI, with torch tensors in
 place of pointers; ``stream`` defaults to torch's current stream):
     attn_fwd(q, k, v, o, lse, causal, scale)
+    attn_fwd_f32(q, k, v, o, lse, causal, scale)   (o in fp32)
     attn_decode_splitkv(q, k, v, o_part, lse_part, num_splits, scale)
     attn_combine(o_part, lse_part, o, lse)
+    attn_merge(o_acc, lse_acc, o_blk, lse_blk, out=None, init=False)
+Ring attention (context parallelism, ``ring.py``): each rank attends its query
+shard to every key/value shard as the shards travel around the ring of ranks,
+merging with attn_merge:
+    ring_attention(q, k, v, causal=False, scale=None, group=None) -> (o, lse)
 Convenience wrappers that allocate the outputs with torch:
     attention(q, k, v, causal=False, scale=None) -> (o, lse)
     decode(q, k, v, scale=None, num_splits=None) -> (o, lse)
@@ -23,9 +29,12 @@ from ._binding import (  # noqa: F401
     attn_decode_splitkv,
     attn_device_status,
     attn_fwd,
+    attn_fwd_f32,
+    attn_merge,
     attn_selftest_bounded_wait,
     attn_status_string,
     decode,
     decode_chunk,
     library_path,
 )
+from .ring import ring_attention, ring_attention_emulated, ring_schedule  # noqa: F401,E402

@@ -32,6 +32,8 @@ def _load():
     P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.attn_fwd.restype = I
+    lib.attn_fwd_f32.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.attn_fwd_f32.restype = I
     lib.attn_decode_splitkv.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.attn_decode_splitkv.restype = I
     lib.attn_combine.argtypes = [P, P, P, P, I, I, I, I, P]
@@ -46,6 +48,8 @@ def _load():
     lib.attn_selftest_bounded_wait.restype = I
     lib.attn_decode_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.attn_decode_noalloc.restype = I
+    lib.attn_merge.argtypes = [P, P, P, P, P, ctypes.c_longlong, I, I, P]
+    lib.attn_merge.restype = I
     return lib
 
 
@@ -97,6 +101,20 @@ def attn_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None):
                          float(scale), _stream(stream)), "attn_fwd")
 
 
+def attn_fwd_f32(q, k, v, o, lse, causal: bool, scale: float, stream=None):
+    """attn_fwd with o [B,Hq,N,d] in fp32 (not rounded to bf16)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    _need(o, torch.float32, "o")
+    _need(lse, torch.float32, "lse")
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape or o.shape != q.shape or lse.shape != (B, Hq, N):
+        raise ValueError("attn_fwd_f32: inconsistent shapes")
+    _check(_lib.attn_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, int(bool(causal)),
+                             float(scale), _stream(stream)), "attn_fwd_f32")
+
+
 def attn_decode_splitkv(q, k, v, o_part, lse_part, num_splits: int, scale: float, stream=None):
     """q [B,Hq,d], k/v [B,Hkv,L,d] bf16; o_part [B,Hq,S,d], lse_part [B,Hq,S] fp32."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -124,6 +142,25 @@ def attn_combine(o_part, lse_part, o, lse, stream=None):
         raise ValueError("attn_combine: inconsistent shapes")
     _check(_lib.attn_combine(_ptr(o_part), _ptr(lse_part), _ptr(o), _ptr(lse), B, Hq, S, d, _stream(stream)),
            "attn_combine")
+
+
+def attn_merge(o_acc, lse_acc, o_blk, lse_blk, out=None, init=False, stream=None):
+    """Folds one block's (o_blk fp32 [..., d], lse_blk fp32 [...]) into the running
+    (o_acc fp32, lse_acc fp32) of the same shape; with `out` (bf16) the merged O
+    goes there instead of into o_acc. Rows = lse_blk.numel()."""
+    _need(o_acc, torch.float32, "o_acc")
+    _need(lse_acc, torch.float32, "lse_acc")
+    _need(o_blk, torch.float32, "o_blk")
+    _need(lse_blk, torch.float32, "lse_blk")
+    if out is not None:
+        _need(out, torch.bfloat16, "out")
+    d = o_blk.shape[-1]
+    rows = lse_blk.numel()
+    if (o_acc.shape != o_blk.shape or lse_acc.shape != lse_blk.shape or o_blk.numel() != rows * d
+            or (out is not None and out.shape != o_blk.shape)):
+        raise ValueError("attn_merge: inconsistent shapes")
+    _check(_lib.attn_merge(_ptr(o_acc), _ptr(lse_acc), _ptr(o_blk), _ptr(lse_blk), _ptr(out), rows, d,
+                           1 if init else 0, _stream(stream)), "attn_merge")
 
 
 def attn_decode_default_splits(B: int, Hq: int, Hkv: int, L: int) -> int:

@@ -16,6 +16,7 @@
 #include "../../include/attn.h"
 #include "attn_fwd_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "merge_sm100.cuh"
 
 namespace eab {
 namespace {
@@ -57,11 +58,11 @@ bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool F32OUT>
 attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                          cudaStream_t stream) {
     using C = FwdCfg<D>;
-    auto kern = attn_fwd_kernel<D, CAUSAL>;
+    auto kern = attn_fwd_kernel<D, CAUSAL, F32OUT>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
     // persistent grid: one CTA per SM, each walking its share of the work items
@@ -107,6 +108,34 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
     mbar_wait(&bar, 0, &abort_flag, limit_ns);
 }
 
+template <bool F32OUT>
+attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                       int N, int d, int causal, float scale, attn_stream_t stream) {
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return ATTN_ERR_INVALID_ARG;
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || (causal != 0 && causal != 1) || !scale_ok(scale))
+        return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (static_cast<long long>(B) * Hq > 65535LL * 1024) return ATTN_ERR_INVALID_ARG;
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, q, d, N, B * Hq, 128) || !make_map(&tk, k, d, N, B * Hkv, 128) ||
+        !make_map(&tv, v, d, N, B * Hkv, 128))
+        return ATTN_ERR_CUDA;
+    FwdParams p;
+    p.o = o;
+    p.lse = lse;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N;
+    p.n_qblocks = (N + 255) / 256;
+    const long long items = static_cast<long long>(p.n_qblocks) * B * Hq;
+    if (items > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    p.n_items = static_cast<int>(items);
+    p.scale_log2 = scale * kLog2e;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 128)
+        return causal ? launch_fwd<128, true, F32OUT>(tq, tk, tv, p, st) : launch_fwd<128, false, F32OUT>(tq, tk, tv, p, st);
+    return causal ? launch_fwd<64, true, F32OUT>(tq, tk, tv, p, st) : launch_fwd<64, false, F32OUT>(tq, tk, tv, p, st);
+}
+
 }  // namespace
 }  // namespace eab
 
@@ -127,28 +156,12 @@ const char* attn_status_string(attn_status_t s) {
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                        int N, int d, int causal, float scale, attn_stream_t stream) {
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
-        return ATTN_ERR_INVALID_ARG;
-    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || (causal != 0 && causal != 1) || !scale_ok(scale))
-        return ATTN_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-    if (static_cast<long long>(B) * Hq > 65535LL * 1024) return ATTN_ERR_INVALID_ARG;
-    CUtensorMap tq, tk, tv;
-    if (!make_map(&tq, q, d, N, B * Hq, 128) || !make_map(&tk, k, d, N, B * Hkv, 128) ||
-        !make_map(&tv, v, d, N, B * Hkv, 128))
-        return ATTN_ERR_CUDA;
-    FwdParams p;
-    p.o = static_cast<__nv_bfloat16*>(o);
-    p.lse = lse;
-    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N;
-    p.n_qblocks = (N + 255) / 256;
-    const long long items = static_cast<long long>(p.n_qblocks) * B * Hq;
-    if (items > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-    p.n_items = static_cast<int>(items);
-    p.scale_log2 = scale * kLog2e;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (d == 128) return causal ? launch_fwd<128, true>(tq, tk, tv, p, st) : launch_fwd<128, false>(tq, tk, tv, p, st);
-    return causal ? launch_fwd<64, true>(tq, tk, tv, p, st) : launch_fwd<64, false>(tq, tk, tv, p, st);
+    return fwd_impl<false>(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream);
+}
+
+attn_status_t attn_fwd_f32(const void* q, const void* k, const void* v, float* o, float* lse, int B, int Hq,
+                           int Hkv, int N, int d, int causal, float scale, attn_stream_t stream) {
+    return fwd_impl<true>(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream);
 }
 
 attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
@@ -190,6 +203,23 @@ attn_status_t attn_combine(const float* o_part, const float* lse_part, void* o, 
         combine_kernel<128><<<static_cast<unsigned>(blocks), 128, smem, st>>>(o_part, lse_part, ob, lse, num_splits);
     else
         combine_kernel<64><<<static_cast<unsigned>(blocks), 64, smem, st>>>(o_part, lse_part, ob, lse, num_splits);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_merge(float* o_acc, float* lse_acc, const float* o_blk, const float* lse_blk, void* out,
+                         long long rows, int d, int init, attn_stream_t stream) {
+    if (!aligned16(o_acc) || !aligned16(lse_acc) || !aligned16(o_blk) || !aligned16(lse_blk)) return ATTN_ERR_INVALID_ARG;
+    if (out != nullptr && !aligned16(out)) return ATTN_ERR_INVALID_ARG;
+    if (rows < 1) return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    const long long blocks = (rows + 7) / 8;  // one warp per row, 8 rows per block
+    if (blocks > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    auto* outb = static_cast<__nv_bfloat16*>(out);
+    if (d == 128)
+        merge_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(o_acc, lse_acc, o_blk, lse_blk, outb, rows, init);
+    else
+        merge_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(o_acc, lse_acc, o_blk, lse_blk, outb, rows, init);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -54,7 +54,7 @@
 namespace eab {
 
 struct FwdParams {
-    __nv_bfloat16* o;  // [B, Hq, N, D]
+    void* o;           // [B, Hq, N, D]: bf16, or fp32 for the F32OUT kernels
     float* lse;        // [B, Hq, N]
     int B, Hq, Hkv, N;
     int n_qblocks;     // ceil(N / 256)
@@ -126,7 +126,7 @@ __device__ __forceinline__ float max64(const float (&v)[64]) {
     return max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool F32OUT>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -467,6 +467,38 @@ __global__ void __launch_bounds__(384, 1)
             const float inv_l = 1.f / l;
             uint8_t* stage = sO + warp * C::STAGE_O_BYTES;
             const int row0 = item.qb * 2 * BM + t * BM + quad * 32;  // first row of this warp
+            if constexpr (F32OUT) {
+                // fp32 O, 32 columns (128 bytes of a row) at a time; chunk i of row
+                // r sits at slot i ^ (r & 7) of the staging buffer
+                float* of = static_cast<float*>(p.o);
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r3[32];
+                    tmem_ld32(o_addr + c * 32, r3);
+                    if (c == D / 32 - 1) {
+                        // O_t is in registers: the next item's first P V may overwrite it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&o_free[t]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        *reinterpret_cast<float4*>(stage + lane * 128 + ((i ^ (lane & 7)) << 4)) =
+                            make_float4(__uint_as_float(r3[4 * i + 0]) * inv_l, __uint_as_float(r3[4 * i + 1]) * inv_l,
+                                        __uint_as_float(r3[4 * i + 2]) * inv_l, __uint_as_float(r3[4 * i + 3]) * inv_l);
+                    __syncwarp();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int rr = 4 * k + (lane >> 3), chunk = lane & 7;
+                        const float4 v4 = *reinterpret_cast<const float4*>(stage + rr * 128 + ((chunk ^ (rr & 7)) << 4));
+                        if (row0 + rr < p.N)
+                            *reinterpret_cast<float4*>(of + (static_cast<size_t>(item.bh) * p.N + row0 + rr) * D +
+                                                       c * 32 + chunk * 4) = v4;
+                    }
+                    __syncwarp();
+                }
+            } else {
+            __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(p.o);
 #pragma unroll
             for (int half = 0; half < D / 64; ++half) {
                 // this lane's row, columns [64*half, 64*half + 64): 128 bytes as 8
@@ -500,10 +532,11 @@ __global__ void __launch_bounds__(384, 1)
                     const int rr = 4 * k + (lane >> 3), chunk = lane & 7;
                     const uint4 v4 = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((chunk ^ (rr & 7)) << 4));
                     if (row0 + rr < p.N)
-                        *reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(item.bh) * p.N + row0 + rr) * D +
+                        *reinterpret_cast<uint4*>(ob + (static_cast<size_t>(item.bh) * p.N + row0 + rr) * D +
                                                   half * 64 + chunk * 8) = v4;
                 }
                 __syncwarp();
+            }
             }
             if (grow < p.N)
                 p.lse[static_cast<size_t>(item.bh) * p.N + grow] = (m_used + log2f(l)) * 0.69314718055994530942f;

@@ -66,6 +66,18 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                        attn_stream_t stream);
 
 /*
+ * attn_fwd_f32 — attn_fwd with O written in fp32 (O_acc / l, not rounded to
+ * bf16): the form a partial result takes when it is merged further, e.g. one
+ * key/value block of ring attention folded in with attn_merge. Same method,
+ * arguments, layouts, checks and errors as attn_fwd except
+ *  o  [B, Hq, N, d] fp32 (device, written).
+ * bf16(o of attn_fwd_f32) with round-to-nearest-even equals o of attn_fwd.
+ */
+attn_status_t attn_fwd_f32(const void* q, const void* k, const void* v, float* o, float* lse,
+                           int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                           attn_stream_t stream);
+
+/*
  * attn_decode_splitkv — split-KV (Flash-Decoding) partials for one query token.
  * Defined by: FlashAttention V2 page, Flash-Decoding paragraph (the key/value
  * sequence is split across thread blocks for single-query decode); each split is
@@ -99,6 +111,33 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v,
  */
 attn_status_t attn_combine(const float* o_part, const float* lse_part, void* o, float* lse,
                            int B, int Hq, int num_splits, int d, attn_stream_t stream);
+
+/*
+ * attn_merge — folds the attention of one key/value block into a running result:
+ * the merge step of ring attention (context parallelism), where the key/value
+ * shards of a long sequence travel around a ring of devices and each device
+ * attends its query shard to every shard in turn, one attn_fwd per shard.
+ * Defined by: FlashAttention-3 page (attention over a key range split into parts
+ * is the log-sum-exp weighted merge of the parts: its split-K combine and the
+ * RingAttention derivation it refers to). Blocks come in fp32 so that a ring
+ * rounds its result to bf16 once, at the last merge. Per row, with
+ * M = max(lse_acc, lse_blk),
+ * wa = exp(lse_acc - M), wb = exp(lse_blk - M):
+ *   o_acc <- (wa o_acc + wb o_blk) / (wa + wb),   lse_acc <- M + ln(wa + wb);
+ * a side whose lse is -inf has weight 0; a row with both -inf is left as it was.
+ *
+ *  o_acc   [rows, d] fp32 (device): read unless init; written unless out is given
+ *  lse_acc [rows]    fp32 (device): read unless init; always written
+ *  o_blk   [rows, d] fp32 (device, read): e.g. the o of attn_fwd_f32, rows = B*Hq*N
+ *  lse_blk [rows]    fp32 (device, read): the matching lse
+ *  out     [rows, d] bf16 (device, written) or NULL: when given, the merged O is
+ *          written here (bf16, round to nearest even) instead of into o_acc —
+ *          the last merge of a ring
+ *  init    nonzero: o_acc and lse_acc are not read; the result is the block itself
+ *  rows >= 1; d 64 or 128. o_acc, out and o_blk must not overlap.
+ */
+attn_status_t attn_merge(float* o_acc, float* lse_acc, const float* o_blk, const float* lse_blk,
+                         void* out, long long rows, int d, int init, attn_stream_t stream);
 
 /*
  * attn_decode_default_splits — the split count attn_decode_splitkv is tuned for

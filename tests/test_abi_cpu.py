@@ -51,6 +51,12 @@ def _fwd(lib, q=16, k=32, v=48, o=64, lse=80, B=1, Hq=2, Hkv=1, N=8, d=64, causa
     return lib.attn_fwd(P(q), P(k), P(v), P(o), P(lse), B, Hq, Hkv, N, d, causal, ctypes.c_float(scale), None)
 
 
+def _fwd32(lib, q=16, k=32, v=48, o=64, lse=80, B=1, Hq=2, Hkv=1, N=8, d=64, causal=0, scale=0.125):
+    P = ctypes.c_void_p
+    lib.attn_fwd_f32.restype = ctypes.c_int
+    return lib.attn_fwd_f32(P(q), P(k), P(v), P(o), P(lse), B, Hq, Hkv, N, d, causal, ctypes.c_float(scale), None)
+
+
 def _dec(lib, q=16, k=32, v=48, op=64, lp=80, B=1, Hq=4, Hkv=2, L=100, d=128, S=4, scale=0.1):
     P = ctypes.c_void_p
     lib.attn_decode_splitkv.restype = ctypes.c_int
@@ -72,6 +78,16 @@ INVALID, UNSUPPORTED = 1, 2
                                 dict(scale=float("nan"))])
 def test_fwd_rejects_invalid(lib, kw):
     assert _fwd(lib, **kw) == INVALID
+
+
+@pytest.mark.parametrize("kw", [dict(q=0), dict(o=0), dict(o=24), dict(N=0), dict(Hq=3, Hkv=2), dict(causal=2),
+                                dict(scale=0.0)])
+def test_fwd_f32_rejects_invalid(lib, kw):
+    assert _fwd32(lib, **kw) == INVALID
+
+
+def test_fwd_f32_rejects_unsupported_head_dim(lib):
+    assert _fwd32(lib, d=96) == UNSUPPORTED
 
 
 @pytest.mark.parametrize("d", [0, 8, 32, 96, 256])
@@ -96,6 +112,24 @@ def test_combine_rejects_invalid(lib, kw):
 
 def test_combine_rejects_unsupported_head_dim(lib):
     assert _comb(lib, d=100) == UNSUPPORTED
+
+
+def _merge(lib, oa=16, la=32, ob=48, lb=64, out=0, rows=8, d=128, init=0):
+    P = ctypes.c_void_p
+    lib.attn_merge.restype = ctypes.c_int
+    lib.attn_merge.argtypes = [P, P, P, P, P, ctypes.c_longlong, ctypes.c_int, ctypes.c_int, P]
+    return lib.attn_merge(P(oa), P(la), P(ob), P(lb), P(out) if out else None, rows, d, init, None)
+
+
+@pytest.mark.parametrize("kw", [dict(oa=0), dict(la=0), dict(ob=0), dict(lb=0), dict(oa=20), dict(lb=36),
+                                dict(out=40), dict(rows=0), dict(rows=-5), dict(rows=1 << 40)])
+def test_merge_rejects_invalid(lib, kw):
+    assert _merge(lib, **kw) == INVALID
+
+
+@pytest.mark.parametrize("d", [0, 32, 96, 256])
+def test_merge_rejects_unsupported_head_dim(lib, d):
+    assert _merge(lib, d=d) == UNSUPPORTED
 
 
 def test_status_strings(lib):
