@@ -8,7 +8,9 @@
  * inner loop, normalisation once at the end). Single-query decode splits the
  * key range across thread blocks and merges the partial results by their
  * log-sum-exp (FlashAttention V2 page, Flash-Decoding paragraph; FlashAttention-3
- * page, the split-K combine step).
+ * page, the split-K combine step). Ring attention (context parallelism) shards a
+ * long sequence across devices and merges each device's per-shard results the
+ * same way (attn_fwd_f32, attn_merge; FlashAttention-3 page, RingAttention).
  *
  * Conventions shared by every call:
  *  - All tensors are dense, contiguous, row-major device buffers owned by the
