@@ -51,8 +51,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch from one ncu capture, valid only for the kernel source
 # it was taken on (sha256 of the kernel file, first 16 hex digits).
 NCU_TRAFFIC = {
-    # decode_splitkv_kernel<128,4>, B1 Hq32 Hkv8 L131072 d128 (the bench's decode workload)
-    "decode": {"bytes_per_launch": 536985088 + 4048128, "source_sha": "67c9877f6eecc387"},
+    # decode_splitkv_kernel<128>, B1 Hq32 Hkv8 L131072 d128 (the bench's decode workload)
+    "decode": {"bytes_per_launch": 536931840 + 3522304, "source_sha": "47462cbad1d67d1c"},
     # attn_fwd_kernel<128,causal / non-causal>, B2 H32 N2048 d128 (the bench's prefill workloads),
     # read + write with cold caches (ncu flushes them before each captured launch)
     "attn_fwd_causal": {"bytes_per_launch": 148234496 + 16394240, "source_sha": "ed115c8fd1b2acdf"},
@@ -288,7 +288,7 @@ def run_ours(args):
     roof_fwd_nc = {"kernel": "attn_fwd_kernel<128,noncausal>", "bound": "tensor", "achieved": round(tflops_n, 1),
                    "peak": tc_peak, "unit": "TFLOP/s", "frac": round(tflops_n / tc_peak, 4),
                    "traffic": traffic("attn_fwd_noncausal", fwd_sha), "ms": round(t_fwd_n, 5)}
-    roof_dec = {"kernel": "decode_splitkv_kernel<128,4>", "bound": "hbm", "achieved": round(dec_kernel_gbs, 1),
+    roof_dec = {"kernel": "decode_splitkv_kernel<128>", "bound": "hbm", "achieved": round(dec_kernel_gbs, 1),
                 "peak": hbm_peak, "unit": "GB/s", "frac": round(dec_kernel_gbs / hbm_peak, 4),
                 "traffic": traffic("decode", dec_sha), "ms": round(t_dec, 5),
                 "peak_source": f"{peak_src} hbm_gbs"}

@@ -177,9 +177,9 @@ def attn_selftest_bounded_wait(limit_us: int, stream=None):
 
 
 def decode_chunk(L: int, num_splits: int) -> int:
-    """Keys per split used by attn_decode_splitkv: 96 * ceil(ceil(L / S) / 96)."""
+    """Keys per split used by attn_decode_splitkv: 128 * ceil(ceil(L / S) / 128)."""
     per = -(-L // num_splits)
-    return -(-per // 96) * 96
+    return -(-per // 128) * 128
 
 
 # ------------------------------------------------------------- convenience --

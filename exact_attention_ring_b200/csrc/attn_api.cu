@@ -75,27 +75,15 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D, int GH>
-attn_status_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
-                            cudaStream_t stream) {
-    using C = DecCfg<D, GH>;
-    auto kern = decode_splitkv_kernel<D, GH>;
+template <int D>
+attn_status_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream) {
+    using C = DecCfg<D>;
+    auto kern = decode_splitkv_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
     const dim3 grid(p.S, p.Hkv * p.groups, p.B);
     kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
-}
-
-template <int D>
-attn_status_t launch_decode_d(const CUtensorMap& tk, const CUtensorMap& tv, DecodeParams p, cudaStream_t stream) {
-    const int G = p.Hq / p.Hkv;
-    // heads per block: the largest of 4, 2, 1 that divides the group (the query
-    // heads live in registers; more than 4 heads of 128 columns would spill)
-    if (G % 4 == 0) { p.groups = G / 4; return launch_decode<D, 4>(tk, tv, p, stream); }
-    if (G % 2 == 0) { p.groups = G / 2; return launch_decode<D, 2>(tk, tv, p, stream); }
-    p.groups = G;
-    return launch_decode<D, 1>(tk, tv, p, stream);
 }
 
 // One thread waits on an mbarrier that nothing completes, with a short limit.
@@ -175,18 +163,20 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, f
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (B > 65535 || num_splits > 0x7fffffff / 2) return ATTN_ERR_INVALID_ARG;
     const int per = (L + num_splits - 1) / num_splits;
-    const int chunk = (per + 95) / 96 * 96;  // whole 96-key stages
+    const int chunk = (per + 127) / 128 * 128;  // whole 128-key tiles
     CUtensorMap tk, tv;
-    if (!make_map(&tk, k, d, L, B * Hkv, 96) || !make_map(&tv, v, d, L, B * Hkv, 96)) return ATTN_ERR_CUDA;
+    if (!make_map(&tk, k, d, L, B * Hkv, 128) || !make_map(&tv, v, d, L, B * Hkv, 128)) return ATTN_ERR_CUDA;
     DecodeParams p;
     p.q = static_cast<const __nv_bfloat16*>(q);
     p.o_part = o_part;
     p.lse_part = lse_part;
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.S = num_splits; p.chunk = chunk;
-    p.groups = 1;
+    p.G = Hq / Hkv;
+    p.groups = (p.G + 127) / 128;  // query heads of a KV head, 128 rows per block
+    if (static_cast<long long>(Hkv) * p.groups > 65535) return ATTN_ERR_INVALID_ARG;
     p.scale_log2 = scale * kLog2e;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    return d == 128 ? launch_decode_d<128>(tk, tv, p, st) : launch_decode_d<64>(tk, tv, p, st);
+    return d == 128 ? launch_decode<128>(tk, tv, p, st) : launch_decode<64>(tk, tv, p, st);
 }
 
 attn_status_t attn_combine(const float* o_part, const float* lse_part, void* o, float* lse, int B, int Hq,
@@ -228,12 +218,11 @@ int attn_decode_default_splits(int B, int Hq, int Hkv, int L) {
     // One decode block runs per SM (148 on B200) and streams its split at about
     // the SM's share of HBM bandwidth after a fixed start-up worth ~260 keys.
     // Pick the split count that maximises (busy fraction of the SM waves) x
-    // (streaming fraction chunk / (chunk + 260)).
-    constexpr int kSMs = 148, kStage = 96;
+    // (streaming fraction chunk / (chunk + 260)); splits are whole 128-key tiles.
+    constexpr int kSMs = 148, kStage = 128;
     constexpr double kStartupKeys = 260.0;
     const int G = Hq / Hkv;
-    const int gh = (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
-    const long long units = static_cast<long long>(B) * Hkv * (G / gh);
+    const long long units = static_cast<long long>(B) * Hkv * ((G + 127) / 128);
     const int max_s = static_cast<int>(std::min<long long>((L + kStage - 1) / kStage, 4096));
     int best_s = 1;
     double best = -1.0;

@@ -1,28 +1,29 @@
-// Split-KV single-query decode and the log-sum-exp weighted combine.
+// Split-KV single-query decode on the tensor cores, and the log-sum-exp
+// weighted combine.
 //
 // Flash-Decoding (FlashAttention V2 page): for one query token the key/value
 // range is split across thread blocks so that long caches still fill the GPU;
 // each split produces a normalised partial output and its log-sum-exp, and a
 // second kernel merges them (FlashAttention-3 page, split-K combine).
 //
-// Decode is bound by reading K and V from HBM once (about 4 FLOP per byte), so
-// it runs on the CUDA cores, not the tensor cores. B200 mapping, 256 threads
-// (two warps per SM sub-partition, so every thread may hold up to 255 registers):
-//   warps 6, 7  TMA producers: 96-key K and V tiles of this split into a ring
-//               of shared-memory stages (128-byte swizzle, zero fill past L).
-//               One issuing thread streams TMA boxes one after another, so the
-//               boxes of every stage are split between two threads, and boxes
-//               are large (96 rows, 12 KB) because each box costs about the same
-//               time whatever its size.
-//   warps 0-5   each owns 16 keys of every stage, 8 at a time. Lane =
-//               quarter*8 + key: the lane dots its quarter of the key row with
-//               the GH query heads held in registers (the swizzle makes the 8
-//               keys of a quarter-warp hit distinct banks), the quarters are
-//               summed with two shuffles, the warp keeps its own online-softmax
-//               state (log2 units, exp2), and for O += p v each lane owns D/32
-//               output columns of every head. Products use packed f32x2 FMAs.
-//   end         the six warps' states are merged in shared memory into the
-//               split's partial (O_s / l_s, lse_s).
+// The G = Hq / Hkv query heads that share a key/value head are the rows of one
+// 128-row query tile, so each split is a small attention problem: S = Q K^T over
+// 128-key tiles with tcgen05.mma into TMEM (double buffered: S(j+1) is computed
+// while the softmax works on S(j)), an online softmax per row on the CUDA cores,
+// and O += P V with P from TMEM. The tensor core does the per-element work of
+// reading K and V from shared memory, so a block streams at the rate TMA and
+// HBM deliver rather than at the CUDA cores' instruction rate. Rows past G
+// (other heads, or zeros) ride along in the MMAs; their results are discarded.
+// 224 threads:
+//   warps 0-3   stage the query rows into the swizzled operand layout (zeros
+//               past the group's heads), then softmax and epilogue, warp w for
+//               rows 32w .. 32w+31 (its TMEM lane quadrant); only the first
+//               ceil(rows/32) warps take part in those;
+//   warp 4      MMA issuer: S(0), S(1), PV(0), S(2), PV(1), ...;
+//   warps 5, 6  TMA producers: K and V tiles of the split into a ring of
+//               shared-memory slots, in the order the MMAs consume them
+//               (K_0 K_1 V_0 K_2 V_1 ...); boxes split between the two threads.
+// TMEM columns: S buffers [0, 128) and [128, 256), O [256, 256 + D).
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -33,258 +34,305 @@ struct DecodeParams {
     const __nv_bfloat16* q;  // [B, Hq, D]
     float* o_part;           // [B, Hq, S, D]
     float* lse_part;         // [B, Hq, S]
-    int B, Hq, Hkv, L, S, chunk, groups;  // groups = (Hq/Hkv) / GH; chunk a multiple of TK
+    int B, Hq, Hkv, L, S, chunk;  // chunk: keys per split, a multiple of 128
+    int G, groups;                // G = Hq / Hkv; groups of 128 query heads per KV head
     float scale_log2;
 };
 
-template <int D, int GH>
+template <int D>
 struct DecCfg {
-    static constexpr int TK = 96;       // keys per stage
-    static constexpr int STAGES = (D == 128) ? 4 : 8;
-    static constexpr int WARPS = 6;     // compute warps
-    static constexpr int KPW = TK / WARPS;  // keys per warp per stage (two groups of 8)
+    static constexpr int BM = 128;  // query rows per tile (heads of one KV head)
+    static constexpr int BN = 128;  // keys per tile
     static constexpr int CHUNKS = D / 64;
-    static constexpr int BOX_BYTES = TK * 128;
-    static constexpr int TILE_BYTES = TK * D * 2;
-    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // K tile then V tile
-    static constexpr int BOXES = 2 * CHUNKS;            // boxes per stage
-    static constexpr int QPL = D / 4;   // query elements per lane (one quarter of the row)
-    static constexpr int CPL = D / 32;  // output columns per lane
-    static constexpr int NUM_THREADS = 32 * WARPS + 64;
-    // ring | p[WARPS][8 keys][GH] | m,l [WARPS][GH] | o [WARPS][GH][D] | barriers
-    static constexpr int P_OFF = STAGES * STAGE_BYTES;
-    static constexpr int ML_OFF = P_OFF + WARPS * 8 * GH * 4;
-    static constexpr int O_OFF = ML_OFF + 2 * WARPS * GH * 4;
-    static constexpr int BAR_OFF = O_OFF + WARPS * GH * D * 4;
-    static constexpr int SMEM_BYTES = 1024 + BAR_OFF + 2 * STAGES * 8 + 16;
+    static constexpr int Q_BYTES = BM * D * 2;
+    static constexpr int TILE_BYTES = BN * D * 2;
+    static constexpr int SLOTS = (D == 128) ? 6 : 12;
+    static constexpr int NUM_THREADS = 224;
+    // q_ready, slot_full, slot_empty, s_full[2], p_full[2], o_done[2], drain
+    static constexpr int NUM_BARRIERS = 1 + 2 * SLOTS + 2 + 2 + 2 + 1;
+    static constexpr int SMEM_BYTES = 1024 + Q_BYTES + SLOTS * TILE_BYTES + NUM_BARRIERS * 8 + 16;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 };
 
-// bf16 pair (one 32-bit word) -> two floats, exact.
-__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
-__device__ __forceinline__ float2 bf_pair(uint32_t u) { return make_float2(bf_lo(u), bf_hi(u)); }
+// Position of K_j / V_j in the split's load order (the MMA's consumption order)
+// K_0 K_1 V_0 K_2 V_1 ... K_{n-1} V_{n-2} V_{n-1}; dec_load_kind inverts it.
+__device__ __forceinline__ int dec_kpos(int j) { return j == 0 ? 0 : 2 * j - 1; }
+__device__ __forceinline__ int dec_vpos(int j, int n) { return j == n - 1 ? 2 * n - 1 : 2 * j + 2; }
+__device__ __forceinline__ bool dec_load_kind(int i, int n, int* j) {
+    if (i == 2 * n - 1) { *j = n - 1; return true; }
+    if (i == 0) { *j = 0; return false; }
+    if (i & 1) { *j = (i + 1) >> 1; return false; }
+    *j = (i >> 1) - 1;
+    return true;
+}
 
-template <int D, int GH>
-__global__ void __launch_bounds__(DecCfg<D, GH>::NUM_THREADS, 1)
+template <int D>
+__global__ void __launch_bounds__(224, 1)
     decode_splitkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                          const DecodeParams p) {
-    using C = DecCfg<D, GH>;
-    constexpr int TK = C::TK, STAGES = C::STAGES, WARPS = C::WARPS;
+                     const DecodeParams p) {
+    using C = DecCfg<D>;
+    constexpr int BM = C::BM, BN = C::BN, SLOTS = C::SLOTS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* p_s = reinterpret_cast<float*>(smem + C::P_OFF);
-    float* m_s = reinterpret_cast<float*>(smem + C::ML_OFF);
-    float* l_s = m_s + WARPS * GH;
-    float* o_s = reinterpret_cast<float*>(smem + C::O_OFF);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
-    uint64_t* empty = full + STAGES;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + STAGES);
+    uint8_t* sQ = smem;
+    uint8_t* sKV = smem + C::Q_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + SLOTS * C::TILE_BYTES);
+    uint64_t* q_ready = bars;                  // query rows staged (one arrival per warp 0-3)
+    uint64_t* slot_full = q_ready + 1;         // [SLOTS]
+    uint64_t* slot_empty = slot_full + SLOTS;  // [SLOTS]
+    uint64_t* s_full = slot_empty + SLOTS;     // [2]
+    uint64_t* p_full = s_full + 2;             // [2] (one arrival per softmax warp)
+    // P V(j) completes phase j >> 1 of o_done[j & 1]. One barrier per parity:
+    // S(j) done implies only P V(j-2) done, so a single barrier could be two
+    // phases behind a waiter and its parity test would pass too early.
+    uint64_t* o_done = p_full + 2;
+    uint64_t* drain = o_done + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int split = blockIdx.x;
     const int hk = blockIdx.y / p.groups, grp = blockIdx.y % p.groups;
     const int b = blockIdx.z;
-    const int G = p.Hq / p.Hkv;
-    const int h0 = hk * G + grp * GH;  // first query head of this block
+    const int h0 = hk * p.G + grp * BM;              // first query head of this tile
+    const int rows = min(BM, p.G - grp * BM);        // real query rows
+    const int nsw = (rows + 31) / 32;                // softmax warps taking part
     const int k0 = split * p.chunk;
     const int k1 = min(p.L, k0 + p.chunk);
-    const int ntiles = k1 > k0 ? (k1 - k0 + TK - 1) / TK : 0;
+    const int nt = k1 > k0 ? (k1 - k0 + BN - 1) / BN : 0;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&full[i], C::BOXES);  // one expect_tx arrival per box
-            mbar_init(&empty[i], WARPS);
+        mbar_init(q_ready, 4);
+        for (int i = 0; i < SLOTS; ++i) {
+            mbar_init(&slot_full[i], C::CHUNKS);
+            mbar_init(&slot_empty[i], 1);
         }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], nsw);
+        }
+        mbar_init(&o_done[0], 1);
+        mbar_init(&o_done[1], 1);
+        mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
+    if (warp == 4) {
+        tmem_alloc(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
 
-    if (warp >= WARPS) {
+    if (warp >= 5) {
         // ------------------------------------------------------ producers ---
-        // box x of a stage (x < CHUNKS: K chunk x, else V chunk x - CHUNKS) is
-        // issued by producer x % 2
-        const int me = warp - WARPS;
-        if (lane == 0 && ntiles > 0) {
+        if (lane == 0 && nt > 0) {
+            const int me = warp - 5;
+            constexpr uint32_t BOX_BYTES = BN * 128;
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             const int z = b * p.Hkv + hk;
             int issued = 0;
-            for (int t = 0; t < ntiles; ++t) {
-                const int slot = t % STAGES, use = t / STAGES;
-                if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, abort_flag)) break;
-                uint8_t* dst = smem + slot * C::STAGE_BYTES;
+            for (int i = 0; i < 2 * nt; ++i) {
+                bool mine = false;
 #pragma unroll
-                for (int x = 0; x < C::BOXES; ++x) {
-                    if (x % 2 != me) continue;
-                    const int c = x % C::CHUNKS;
-                    const bool is_v = x >= C::CHUNKS;
-                    mbar_arrive_expect_tx(&full[slot], C::BOX_BYTES);
-                    tma_load_3d(dst + (is_v ? C::TILE_BYTES : 0) + c * C::BOX_BYTES, is_v ? &tm_v : &tm_k,
-                                &full[slot], c * 64, k0 + t * TK, z);
+                for (int c = 0; c < C::CHUNKS; ++c) mine |= ((i * C::CHUNKS + c) & 1) == me;
+                if (!mine) continue;
+                const int slot = i % SLOTS, use = i / SLOTS;
+                if (use > 0 && !mbar_wait(&slot_empty[slot], (use - 1) & 1, abort_flag)) break;
+                int j;
+                const CUtensorMap* tm = dec_load_kind(i, nt, &j) ? &tm_v : &tm_k;
+                uint8_t* dst = sKV + slot * C::TILE_BYTES;
+#pragma unroll
+                for (int c = 0; c < C::CHUNKS; ++c) {
+                    if (((i * C::CHUNKS + c) & 1) != me) continue;
+                    mbar_arrive_expect_tx(&slot_full[slot], BOX_BYTES);
+                    tma_load_3d(dst + c * BOX_BYTES, tm, &slot_full[slot], c * 64, k0 + j * BN, z);
                 }
-                issued = t + 1;
+                issued = i + 1;
             }
-            for (int t = max(0, issued - STAGES); t < issued; ++t)
-                mbar_wait(&full[t % STAGES], (t / STAGES) & 1, nullptr);
+            // Let every copy in flight land before the CTA can exit.
+            for (int i = max(0, issued - SLOTS); i < issued; ++i)
+                mbar_wait(&slot_full[i % SLOTS], (i / SLOTS) & 1, nullptr);
         }
-        return;  // producers take no part in the merge below (named barrier 1 counts the compute warps)
-    }
-
-    // -------------------------------------------------------- compute -------
-    const int qtr = lane >> 3;  // quarter of the key row this lane dots
-    const int kk = lane & 7;    // key of the current group of 8 this lane owns
-    float2 qreg[GH][C::QPL / 2];
+    } else if (warp == 4) {
+        // ---------------------------------------------------- MMA issuer ----
+        if (lane == 0 && nt > 0) {
+            constexpr uint32_t idesc_qk = make_idesc_bf16(BM, BN, 0, 0);
+            constexpr uint32_t idesc_pv = make_idesc_bf16(BM, D, 0, 1);
+            const uint32_t o_tmem = tmem + 256;
+            const uint32_t q_addr = smem_addr(sQ), kv_addr = smem_addr(sKV);
+            bool ok = mbar_wait(q_ready, 0, abort_flag);
+            auto issue_s = [&](int j) -> bool {
+                const int ik = dec_kpos(j);
+                if (!mbar_wait(&slot_full[ik % SLOTS], (ik / SLOTS) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t k_addr = kv_addr + (ik % SLOTS) * C::TILE_BYTES;
+                const uint32_t s_tmem = tmem + (j & 1) * 128;
 #pragma unroll
-    for (int g = 0; g < GH; ++g) {
-        const __nv_bfloat16* qrow = p.q + (static_cast<size_t>(b) * p.Hq + h0 + g) * D + qtr * C::QPL;
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk & 3) * 32;
+                    const uint64_t ad = make_sdesc_sw128(q_addr + (kk >> 2) * (BM * 128) + koff, 16, 1024);
+                    const uint64_t bd = make_sdesc_sw128(k_addr + (kk >> 2) * (BN * 128) + koff, 16, 1024);
+                    mma_ss(s_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(&s_full[j & 1]);
+                tc_commit(&slot_empty[ik % SLOTS]);
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            if (ok && nt > 1) ok = issue_s(1);
+            for (int j = 0; ok && j < nt; ++j) {
+                // O += P(j) V_j, then S(j+2) into the S buffer this product reads
+                const int iv = dec_vpos(j, nt);
+                ok = mbar_wait(&slot_full[iv % SLOTS], (iv / SLOTS) & 1, abort_flag) &&
+                     mbar_wait_spin(&p_full[j & 1], (j >> 1) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t v_addr = kv_addr + (iv % SLOTS) * C::TILE_BYTES;
+                const uint32_t p_tmem = tmem + (j & 1) * 128;
 #pragma unroll
-        for (int i = 0; i < C::QPL; i += 8) {
-            const uint4 u = *reinterpret_cast<const uint4*>(qrow + i);
-            qreg[g][i / 2 + 0] = bf_pair(u.x);
-            qreg[g][i / 2 + 1] = bf_pair(u.y);
-            qreg[g][i / 2 + 2] = bf_pair(u.z);
-            qreg[g][i / 2 + 3] = bf_pair(u.w);
-        }
-    }
-    float m[GH], lsum[GH];
-    float2 acc[GH][C::CPL / 2];
-#pragma unroll
-    for (int g = 0; g < GH; ++g) {
-        m[g] = -INFINITY;
-        lsum[g] = 0.f;
-#pragma unroll
-        for (int e = 0; e < C::CPL / 2; ++e) acc[g][e] = make_float2(0.f, 0.f);
-    }
-    float* pw = p_s + warp * 8 * GH;
-
-    for (int t = 0; t < ntiles; ++t) {
-        const int slot = t % STAGES;
-        const bool w = mbar_wait(&full[slot], (t / STAGES) & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, w)) break;
-        const uint8_t* sK = smem + slot * C::STAGE_BYTES;
-        const uint8_t* sV = sK + C::TILE_BYTES;
-#pragma unroll
-        for (int sub = 0; sub < C::KPW / 8; ++sub) {
-            const int r = warp * C::KPW + sub * 8 + kk;  // row of this lane's key inside the stage
-            // scores: this lane's quarter of key r against the GH query heads
-            float2 part[GH];
-#pragma unroll
-            for (int g = 0; g < GH; ++g) part[g] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int i = 0; i < C::QPL / 8; ++i) {
-                const int cc = qtr * (C::QPL / 8) + i;  // logical 16-byte chunk in the row
-                const uint4 u = *reinterpret_cast<const uint4*>(sK + (cc >> 3) * C::BOX_BYTES + r * 128 +
-                                                                (((cc & 7) ^ (r & 7)) << 4));
-                const float2 kf[4] = {bf_pair(u.x), bf_pair(u.y), bf_pair(u.z), bf_pair(u.w)};
-#pragma unroll
-                for (int g = 0; g < GH; ++g)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) part[g] = ffma2(qreg[g][i * 4 + e], kf[e], part[g]);
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint64_t bd = make_sdesc_sw128(v_addr + kk * 16 * 128, BN * 128, 1024);
+                    mma_ts(o_tmem, p_tmem + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(&o_done[j & 1]);
+                tc_commit(&slot_empty[iv % SLOTS]);
+                if (j + 2 < nt) ok = issue_s(j + 2);
             }
-            const bool valid = k0 + t * TK + r < k1;
-            float pr[GH];
+            // Every MMA must be complete before TMEM is released.
+            tc_commit(drain);
+            mbar_wait(drain, 0, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------- query staging, softmax ----
+        const int row = warp * 32 + lane;
+        const bool real = row < rows;
+        const size_t out_row = static_cast<size_t>(b) * p.Hq + h0 + row;
+        if (nt > 0) {
+            // this warp's 32 query rows in the K-major 128-byte-swizzled operand
+            // layout (rows past the group's heads as zeros)
 #pragma unroll
-            for (int g = 0; g < GH; ++g) {
-                float sdot = part[g].x + part[g].y;
-                sdot += __shfl_xor_sync(0xffffffffu, sdot, 8);
-                sdot += __shfl_xor_sync(0xffffffffu, sdot, 16);
-                const float s2 = valid ? sdot * p.scale_log2 : -INFINITY;
-                float tmax = s2;
-                tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
-                tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
-                tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
-                const float m_new = fmaxf(m[g], tmax);
-                const float factor = (m_new == m[g]) ? 1.f : ex2_approx(m[g] - m_new);
-                m[g] = m_new;
-                lsum[g] *= factor;
-                if (factor != 1.f) {
+            for (int c = 0; c < D / 8; ++c) {
+                uint4 v4 = make_uint4(0u, 0u, 0u, 0u);
+                if (real) v4 = *reinterpret_cast<const uint4*>(p.q + out_row * D + c * 8);
+                *reinterpret_cast<uint4*>(sQ + (c >> 3) * (BM * 128) + row * 128 + (((c & 7) ^ (row & 7)) << 4)) = v4;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_ready);
+        }
+        if (warp >= nsw) {
+            // no real rows in this quadrant
+        } else if (nt == 0) {
+            // an empty split: weight 0 in the combine
+            if (real) {
+                p.lse_part[out_row * p.S + split] = -INFINITY;
+#pragma unroll 4
+                for (int c = 0; c < D; c += 4)
+                    *reinterpret_cast<float4*>(p.o_part + (out_row * p.S + split) * D + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        } else {
+            const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
+            const uint32_t o_addr = lane_base + 256;
+            const float c2 = p.scale_log2;
+            float m_used = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int j = 0; j < nt; ++j) {
+                const uint32_t s_addr = lane_base + (j & 1) * 128;
+                const bool w1 = mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag);
+                if (!__all_sync(0xffffffffu, w1)) { ok = false; break; }
+                tc_fence_after();
+                const int lim = min(BN, k1 - (k0 + j * BN));  // valid keys of this tile
+                float mx = -INFINITY;
+                uint32_t sv[128];
 #pragma unroll
-                    for (int e = 0; e < C::CPL / 2; ++e) {
-                        acc[g][e].x *= factor;
-                        acc[g][e].y *= factor;
+                for (int h = 0; h < 2; ++h) {
+                    tmem_ld64(s_addr + h * 64, reinterpret_cast<uint32_t(&)[64]>(sv[h * 64]));
+                }
+                if (lim < BN) {
+#pragma unroll
+                    for (int i = 0; i < 128; ++i)
+                        if (i >= lim) sv[i] = 0xff800000u;  // -inf: exp2 gives 0
+                }
+#pragma unroll
+                for (int i = 0; i < 128; i += 2) mx = max3(mx, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+                const float m_tile = mx * c2;
+                const bool need = m_tile > m_used + C::RESCALE_THRESHOLD;
+                float factor = 1.f;
+                if (need) {
+                    factor = ex2_approx(m_used - m_tile);
+                    m_used = m_tile;
+                }
+                l *= factor;
+                if (j > 0 && __any_sync(0xffffffffu, need)) {
+                    // O must hold P V(j-1) before it is rescaled (S(j) implies only P V(j-2))
+                    const bool w3 = mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag);
+                    if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t r3[32];
+                        tmem_ld32(o_addr + c * 32, r3);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r3[i] = __float_as_uint(__uint_as_float(r3[i]) * factor);
+                        tmem_st32(o_addr + c * 32, r3);
                     }
                 }
-                const float m_safe = (m_new == -INFINITY) ? 0.f : m_new;
-                pr[g] = ex2_approx(s2 - m_safe);
-                if (qtr == 0) lsum[g] += pr[g];
-            }
-            if (qtr == 0) {
+                const float2 c2x2 = make_float2(c2, c2), negm2 = make_float2(-m_used, -m_used);
+                float2 rsum[4];
 #pragma unroll
-                for (int g = 0; g < GH; ++g) pw[kk * GH + g] = pr[g];
-            }
-            __syncwarp();
-            // O += p v over the group's 8 keys; lane owns columns [lane*CPL, lane*CPL+CPL)
+                for (int k = 0; k < 4; ++k) rsum[k] = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int k2 = 0; k2 < 8; ++k2) {
-                const int r2 = warp * C::KPW + sub * 8 + k2;
-                const int byte = lane * C::CPL * 2;  // byte offset of this lane's columns in the row
-                const int cc = byte >> 4;
-                const uint8_t* src =
-                    sV + (cc >> 3) * C::BOX_BYTES + r2 * 128 + ((((cc & 7) ^ (r2 & 7)) << 4) | (byte & 15));
-                float2 vf[C::CPL / 2];
-                if constexpr (C::CPL == 4) {
-                    const uint2 u = *reinterpret_cast<const uint2*>(src);
-                    vf[0] = bf_pair(u.x);
-                    vf[1] = bf_pair(u.y);
-                } else {
-                    vf[0] = bf_pair(*reinterpret_cast<const uint32_t*>(src));
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int e = h * 64 + 2 * i;
+                        const float2 y = ffma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2x2, negm2);
+                        const float2 pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+                        rsum[i & 3] = fadd2(rsum[i & 3], pp);
+                        pk[i] = pack_bf16x2(pp.x, pp.y);
+                    }
+                    tmem_st32(s_addr + h * 32, pk);
                 }
-#pragma unroll
-                for (int g = 0; g < GH; ++g) {
-                    const float pg = pw[k2 * GH + g];
-                    const float2 pp = make_float2(pg, pg);
-#pragma unroll
-                    for (int e = 0; e < C::CPL / 2; ++e) acc[g][e] = ffma2(pp, vf[e], acc[g][e]);
-                }
+                const float2 rs = fadd2(fadd2(rsum[0], rsum[1]), fadd2(rsum[2], rsum[3]));
+                l += rs.x + rs.y;
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[j & 1]);
             }
-            __syncwarp();
+            if (ok && __all_sync(0xffffffffu, mbar_wait(&o_done[(nt - 1) & 1], ((nt - 1) >> 1) & 1, abort_flag))) {
+                tc_fence_after();
+                const float inv_l = 1.f / l;
+                float* dst = p.o_part + (out_row * p.S + split) * D;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r3[32];
+                    tmem_ld32(o_addr + c * 32, r3);
+                    if (real) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4*>(dst + c * 32 + i) =
+                                make_float4(__uint_as_float(r3[i]) * inv_l, __uint_as_float(r3[i + 1]) * inv_l,
+                                            __uint_as_float(r3[i + 2]) * inv_l, __uint_as_float(r3[i + 3]) * inv_l);
+                    }
+                }
+                if (real) p.lse_part[out_row * p.S + split] = (m_used + log2f(l)) * 0.69314718055994530942f;
+            }
         }
-        if (lane == 0) mbar_arrive(&empty[slot]);
     }
 
-    // --------------------------------------------- merge the six warps ------
-#pragma unroll
-    for (int g = 0; g < GH; ++g) {
-        float ls = lsum[g];
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
-        if (lane == 0) {
-            m_s[warp * GH + g] = m[g];
-            l_s[warp * GH + g] = ls;
-        }
-    }
-    named_barrier(1, 32 * WARPS);
-#pragma unroll
-    for (int g = 0; g < GH; ++g) {
-        float M = m_s[g];
-#pragma unroll
-        for (int w2 = 1; w2 < WARPS; ++w2) M = fmaxf(M, m_s[w2 * GH + g]);
-        const float f = (m[g] == -INFINITY) ? 0.f : ex2_approx(m[g] - M);
-#pragma unroll
-        for (int e = 0; e < C::CPL / 2; ++e) {
-            o_s[(warp * GH + g) * D + lane * C::CPL + 2 * e] = acc[g][e].x * f;
-            o_s[(warp * GH + g) * D + lane * C::CPL + 2 * e + 1] = acc[g][e].y * f;
-        }
-    }
-    named_barrier(1, 32 * WARPS);
-    const int tid = threadIdx.x;
-    for (int idx = tid; idx < GH * D; idx += 32 * WARPS) {
-        const int g = idx / D, col = idx % D;
-        float M = m_s[g];
-#pragma unroll
-        for (int w2 = 1; w2 < WARPS; ++w2) M = fmaxf(M, m_s[w2 * GH + g]);
-        float Ltot = 0.f, o = 0.f;
-#pragma unroll
-        for (int w2 = 0; w2 < WARPS; ++w2) {
-            const float mw = m_s[w2 * GH + g];
-            Ltot += (mw == -INFINITY) ? 0.f : l_s[w2 * GH + g] * ex2_approx(mw - M);
-            o += o_s[(w2 * GH + g) * D + col];
-        }
-        const size_t u = (static_cast<size_t>(b) * p.Hq + h0 + g) * p.S + split;
-        const bool empty_split = (Ltot == 0.f);
-        p.o_part[u * D + col] = empty_split ? 0.f : o / Ltot;
-        if (col == 0) p.lse_part[u] = empty_split ? -INFINITY : (M + log2f(Ltot)) * 0.69314718055994530942f;
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
     }
 }
 

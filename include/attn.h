@@ -90,7 +90,7 @@ attn_status_t attn_fwd_f32(const void* q, const void* k, const void* v, float* o
  *  o_part   [B, Hq, S, d]   fp32 (device, written): normalised partial outputs
  *  lse_part [B, Hq, S]      fp32 (device, written): natural-log LSE per split
  *  S = num_splits, 1 <= S <= L. Split s covers keys [s*C, min(L, (s+1)*C)) with
- *  C = 96 * ceil(ceil(L / S) / 96). A split with no keys gets lse = -inf, o = 0.
+ *  C = 128 * ceil(ceil(L / S) / 128). A split with no keys gets lse = -inf, o = 0.
  *  d 64 or 128; Hq % Hkv == 0; scale finite and > 0.
  */
 attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v,
@@ -146,7 +146,7 @@ attn_status_t attn_merge(float* o_acc, float* lse_acc, const float* o_blk, const
  * on a 148-SM B200: it maximises the busy fraction of the waves of (batch,
  * kv-head, split) blocks times the fraction of each block's time spent
  * streaming (a block's start-up is worth about 260 keys). Pure host
- * arithmetic; returns 1 <= S <= ceil(L / 96), or 0 on bad arguments.
+ * arithmetic; returns 1 <= S <= ceil(L / 128), or 0 on bad arguments.
  */
 int attn_decode_default_splits(int B, int Hq, int Hkv, int L);
 

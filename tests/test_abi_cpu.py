@@ -159,13 +159,13 @@ def test_default_splits(lib):
     assert f(1, 1, 1, 1) == 1
     for L in (1, 31, 257, 100000):
         s = f(2, 16, 4, L)
-        assert 1 <= s <= -(-L // 96)
+        assert 1 <= s <= -(-L // 128)
 
 
 def test_decode_chunk_rule():
     from exact_attention_ring_b200 import decode_chunk
-    assert decode_chunk(4096, 16) == 288
-    assert decode_chunk(32768, 37) == 960
-    assert decode_chunk(100, 64) == 96
-    assert decode_chunk(1, 1) == 96
-    assert decode_chunk(131072, 5) == 26304
+    assert decode_chunk(4096, 16) == 256
+    assert decode_chunk(32768, 37) == 896
+    assert decode_chunk(100, 64) == 128
+    assert decode_chunk(1, 1) == 128
+    assert decode_chunk(131072, 5) == 26240
