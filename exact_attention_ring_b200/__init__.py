@@ -9,6 +9,7 @@ Low-level calls (same names and arguments as the C ABI, with torch tensors in
 place of pointers; ``stream`` defaults to torch's current stream):
     attn_fwd(q, k, v, o, lse, causal, scale)
     attn_fwd_f32(q, k, v, o, lse, causal, scale)   (o in fp32)
+    attn_fwd_f16, attn_decode_splitkv_f16, attn_combine_f16   (fp16 inputs)
     attn_decode_splitkv(q, k, v, o_part, lse_part, num_splits, scale)
     attn_combine(o_part, lse_part, o, lse)
     attn_merge(o_acc, lse_acc, o_blk, lse_blk, out=None, init=False)
@@ -24,11 +25,14 @@ from ._binding import (  # noqa: F401
     AttnError,
     attention,
     attn_combine,
+    attn_combine_f16,
     attn_decode_default_splits,
     attn_decode_noalloc,
     attn_decode_splitkv,
+    attn_decode_splitkv_f16,
     attn_device_status,
     attn_fwd,
+    attn_fwd_f16,
     attn_fwd_f32,
     attn_merge,
     attn_selftest_bounded_wait,

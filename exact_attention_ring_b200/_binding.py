@@ -34,6 +34,12 @@ def _load():
     lib.attn_fwd.restype = I
     lib.attn_fwd_f32.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.attn_fwd_f32.restype = I
+    lib.attn_fwd_f16.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.attn_fwd_f16.restype = I
+    lib.attn_decode_splitkv_f16.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.attn_decode_splitkv_f16.restype = I
+    lib.attn_combine_f16.argtypes = [P, P, P, P, I, I, I, I, P]
+    lib.attn_combine_f16.restype = I
     lib.attn_decode_splitkv.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.attn_decode_splitkv.restype = I
     lib.attn_combine.argtypes = [P, P, P, P, I, I, I, I, P]
@@ -88,17 +94,26 @@ def _need(t: torch.Tensor, dtype, name: str):
 
 # -------------------------------------------------------------- C ABI calls --
 
-def attn_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None):
-    """q [B,Hq,N,d], k/v [B,Hkv,N,d], o [B,Hq,N,d] bf16; lse [B,Hq,N] fp32."""
+def _fwd(fn, name, dt, q, k, v, o, lse, causal, scale, stream):
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
-        _need(t, torch.bfloat16, n)
+        _need(t, dt, n)
     _need(lse, torch.float32, "lse")
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
     if k.shape != (B, Hkv, N, d) or v.shape != k.shape or o.shape != q.shape or lse.shape != (B, Hq, N):
-        raise ValueError("attn_fwd: inconsistent shapes")
-    _check(_lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, int(bool(causal)),
-                         float(scale), _stream(stream)), "attn_fwd")
+        raise ValueError(f"{name}: inconsistent shapes")
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, int(bool(causal)), float(scale),
+              _stream(stream)), name)
+
+
+def attn_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None):
+    """q [B,Hq,N,d], k/v [B,Hkv,N,d], o [B,Hq,N,d] bf16; lse [B,Hq,N] fp32."""
+    _fwd(_lib.attn_fwd, "attn_fwd", torch.bfloat16, q, k, v, o, lse, causal, scale, stream)
+
+
+def attn_fwd_f16(q, k, v, o, lse, causal: bool, scale: float, stream=None):
+    """attn_fwd for fp16 q, k, v and o."""
+    _fwd(_lib.attn_fwd_f16, "attn_fwd_f16", torch.float16, q, k, v, o, lse, causal, scale, stream)
 
 
 def attn_fwd_f32(q, k, v, o, lse, causal: bool, scale: float, stream=None):
@@ -115,10 +130,9 @@ def attn_fwd_f32(q, k, v, o, lse, causal: bool, scale: float, stream=None):
                              float(scale), _stream(stream)), "attn_fwd_f32")
 
 
-def attn_decode_splitkv(q, k, v, o_part, lse_part, num_splits: int, scale: float, stream=None):
-    """q [B,Hq,d], k/v [B,Hkv,L,d] bf16; o_part [B,Hq,S,d], lse_part [B,Hq,S] fp32."""
+def _dec(fn, name, dt, q, k, v, o_part, lse_part, num_splits, scale, stream):
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, torch.bfloat16, n)
+        _need(t, dt, n)
     _need(o_part, torch.float32, "o_part")
     _need(lse_part, torch.float32, "lse_part")
     B, Hq, d = q.shape
@@ -126,22 +140,42 @@ def attn_decode_splitkv(q, k, v, o_part, lse_part, num_splits: int, scale: float
     S = int(num_splits)
     if k.shape != (B, Hkv, L, d) or v.shape != k.shape or o_part.shape != (B, Hq, S, d) \
             or lse_part.shape != (B, Hq, S):
-        raise ValueError("attn_decode_splitkv: inconsistent shapes")
-    _check(_lib.attn_decode_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), B, Hq, Hkv, L, d,
-                                    S, float(scale), _stream(stream)), "attn_decode_splitkv")
+        raise ValueError(f"{name}: inconsistent shapes")
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), B, Hq, Hkv, L, d, S, float(scale),
+              _stream(stream)), name)
+
+
+def attn_decode_splitkv(q, k, v, o_part, lse_part, num_splits: int, scale: float, stream=None):
+    """q [B,Hq,d], k/v [B,Hkv,L,d] bf16; o_part [B,Hq,S,d], lse_part [B,Hq,S] fp32."""
+    _dec(_lib.attn_decode_splitkv, "attn_decode_splitkv", torch.bfloat16, q, k, v, o_part, lse_part, num_splits,
+         scale, stream)
+
+
+def attn_decode_splitkv_f16(q, k, v, o_part, lse_part, num_splits: int, scale: float, stream=None):
+    """attn_decode_splitkv for fp16 q, k, v."""
+    _dec(_lib.attn_decode_splitkv_f16, "attn_decode_splitkv_f16", torch.float16, q, k, v, o_part, lse_part,
+         num_splits, scale, stream)
+
+
+def _comb(fn, name, dt, o_part, lse_part, o, lse, stream):
+    _need(o_part, torch.float32, "o_part")
+    _need(lse_part, torch.float32, "lse_part")
+    _need(o, dt, "o")
+    _need(lse, torch.float32, "lse")
+    B, Hq, S, d = o_part.shape
+    if lse_part.shape != (B, Hq, S) or o.shape != (B, Hq, d) or lse.shape != (B, Hq):
+        raise ValueError(f"{name}: inconsistent shapes")
+    _check(fn(_ptr(o_part), _ptr(lse_part), _ptr(o), _ptr(lse), B, Hq, S, d, _stream(stream)), name)
 
 
 def attn_combine(o_part, lse_part, o, lse, stream=None):
     """o_part [B,Hq,S,d], lse_part [B,Hq,S] fp32 -> o [B,Hq,d] bf16, lse [B,Hq] fp32."""
-    _need(o_part, torch.float32, "o_part")
-    _need(lse_part, torch.float32, "lse_part")
-    _need(o, torch.bfloat16, "o")
-    _need(lse, torch.float32, "lse")
-    B, Hq, S, d = o_part.shape
-    if lse_part.shape != (B, Hq, S) or o.shape != (B, Hq, d) or lse.shape != (B, Hq):
-        raise ValueError("attn_combine: inconsistent shapes")
-    _check(_lib.attn_combine(_ptr(o_part), _ptr(lse_part), _ptr(o), _ptr(lse), B, Hq, S, d, _stream(stream)),
-           "attn_combine")
+    _comb(_lib.attn_combine, "attn_combine", torch.bfloat16, o_part, lse_part, o, lse, stream)
+
+
+def attn_combine_f16(o_part, lse_part, o, lse, stream=None):
+    """attn_combine with o in fp16."""
+    _comb(_lib.attn_combine_f16, "attn_combine_f16", torch.float16, o_part, lse_part, o, lse, stream)
 
 
 def attn_merge(o_acc, lse_acc, o_blk, lse_blk, out=None, init=False, stream=None):
@@ -185,17 +219,19 @@ def decode_chunk(L: int, num_splits: int) -> int:
 # ------------------------------------------------------------- convenience --
 
 def attention(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
-    """Allocates o, lse and runs attn_fwd. Returns (o bf16, lse fp32)."""
+    """Allocates o, lse and runs attn_fwd (attn_fwd_f16 for fp16 inputs).
+    Returns (o in the input type, lse fp32)."""
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[-1])
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)
-    attn_fwd(q, k, v, o, lse, causal, scale, stream)
+    (attn_fwd_f16 if q.dtype == torch.float16 else attn_fwd)(q, k, v, o, lse, causal, scale, stream)
     return o, lse
 
 
 def decode(q, k, v, scale: float | None = None, num_splits: int | None = None, stream=None):
-    """Split-KV decode plus combine. q [B,Hq,d], k/v [B,Hkv,L,d] -> (o [B,Hq,d], lse [B,Hq])."""
+    """Split-KV decode plus combine (bf16 or fp16 inputs). q [B,Hq,d], k/v [B,Hkv,L,d] ->
+    (o [B,Hq,d] in the input type, lse [B,Hq])."""
     B, Hq, d = q.shape
     Hkv, L = k.shape[1], k.shape[2]
     if scale is None:
@@ -203,10 +239,11 @@ def decode(q, k, v, scale: float | None = None, num_splits: int | None = None, s
     S = num_splits or attn_decode_default_splits(B, Hq, Hkv, L)
     o_part = torch.empty(B, Hq, S, d, device=q.device, dtype=torch.float32)
     lse_part = torch.empty(B, Hq, S, device=q.device, dtype=torch.float32)
-    attn_decode_splitkv(q, k, v, o_part, lse_part, S, scale, stream)
-    o = torch.empty(B, Hq, d, device=q.device, dtype=torch.bfloat16)
+    f16 = q.dtype == torch.float16
+    (attn_decode_splitkv_f16 if f16 else attn_decode_splitkv)(q, k, v, o_part, lse_part, S, scale, stream)
+    o = torch.empty(B, Hq, d, device=q.device, dtype=q.dtype)
     lse = torch.empty(B, Hq, device=q.device, dtype=torch.float32)
-    attn_combine(o_part, lse_part, o, lse, stream)
+    (attn_combine_f16 if f16 else attn_combine)(o_part, lse_part, o, lse, stream)
     return o, lse
 
 

@@ -40,6 +40,12 @@ EncodeTiledFn encode_fn() {
 
 // bf16 tensor viewed as [planes, rows, D] with a {64, box_rows, 1} box and
 // 128-byte swizzle; rows past `rows` read as zero.
+template <class E>
+constexpr CUtensorMapDataType tma_type() {
+    return E::fmt == ElemF16::fmt ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+}
+
+template <class E>
 bool make_map(CUtensorMap* map, const void* base, int D, int rows, int planes, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -47,7 +53,7 @@ bool make_map(CUtensorMap* map, const void* base, int D, int rows, int planes, i
     const cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(D) * 2 * cuuint64_t(rows)};
     const cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    return fn(map, tma_type<E>(), 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -58,11 +64,11 @@ bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int D, bool CAUSAL, bool F32OUT>
+template <int D, bool CAUSAL, bool F32OUT, class E>
 attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                          cudaStream_t stream) {
     using C = FwdCfg<D>;
-    auto kern = attn_fwd_kernel<D, CAUSAL, F32OUT>;
+    auto kern = attn_fwd_kernel<D, CAUSAL, F32OUT, E>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
     // persistent grid: one CTA per SM, each walking its share of the work items
@@ -75,10 +81,10 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D>
+template <int D, class E>
 attn_status_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream) {
     using C = DecCfg<D>;
-    auto kern = decode_splitkv_kernel<D>;
+    auto kern = decode_splitkv_kernel<D, E>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
     const dim3 grid(p.S, p.Hkv * p.groups, p.B);
@@ -96,7 +102,7 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
     mbar_wait(&bar, 0, &abort_flag, limit_ns);
 }
 
-template <bool F32OUT>
+template <bool F32OUT, class E>
 attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                        int N, int d, int causal, float scale, attn_stream_t stream) {
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
@@ -106,8 +112,8 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (static_cast<long long>(B) * Hq > 65535LL * 1024) return ATTN_ERR_INVALID_ARG;
     CUtensorMap tq, tk, tv;
-    if (!make_map(&tq, q, d, N, B * Hq, 128) || !make_map(&tk, k, d, N, B * Hkv, 128) ||
-        !make_map(&tv, v, d, N, B * Hkv, 128))
+    if (!make_map<E>(&tq, q, d, N, B * Hq, 128) || !make_map<E>(&tk, k, d, N, B * Hkv, 128) ||
+        !make_map<E>(&tv, v, d, N, B * Hkv, 128))
         return ATTN_ERR_CUDA;
     FwdParams p;
     p.o = o;
@@ -120,8 +126,55 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
     p.scale_log2 = scale * kLog2e;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d == 128)
-        return causal ? launch_fwd<128, true, F32OUT>(tq, tk, tv, p, st) : launch_fwd<128, false, F32OUT>(tq, tk, tv, p, st);
-    return causal ? launch_fwd<64, true, F32OUT>(tq, tk, tv, p, st) : launch_fwd<64, false, F32OUT>(tq, tk, tv, p, st);
+        return causal ? launch_fwd<128, true, F32OUT, E>(tq, tk, tv, p, st)
+                      : launch_fwd<128, false, F32OUT, E>(tq, tk, tv, p, st);
+    return causal ? launch_fwd<64, true, F32OUT, E>(tq, tk, tv, p, st) : launch_fwd<64, false, F32OUT, E>(tq, tk, tv, p, st);
+}
+
+template <class E>
+attn_status_t decode_impl(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
+                                  int B, int Hq, int Hkv, int L, int d, int num_splits, float scale,
+                                  attn_stream_t stream) {
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part) || !aligned16(lse_part))
+        return ATTN_ERR_INVALID_ARG;
+    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0 || num_splits < 1 || num_splits > L ||
+        !scale_ok(scale))
+        return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (B > 65535 || num_splits > 0x7fffffff / 2) return ATTN_ERR_INVALID_ARG;
+    const int per = (L + num_splits - 1) / num_splits;
+    const int chunk = (per + 127) / 128 * 128;  // whole 128-key tiles
+    CUtensorMap tk, tv;
+    if (!make_map<E>(&tk, k, d, L, B * Hkv, 128) || !make_map<E>(&tv, v, d, L, B * Hkv, 128)) return ATTN_ERR_CUDA;
+    DecodeParams p;
+    p.q = q;
+    p.o_part = o_part;
+    p.lse_part = lse_part;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.S = num_splits; p.chunk = chunk;
+    p.G = Hq / Hkv;
+    p.groups = (p.G + 127) / 128;  // query heads of a KV head, 128 rows per block
+    if (static_cast<long long>(Hkv) * p.groups > 65535) return ATTN_ERR_INVALID_ARG;
+    p.scale_log2 = scale * kLog2e;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    return d == 128 ? launch_decode<128, E>(tk, tv, p, st) : launch_decode<64, E>(tk, tv, p, st);
+}
+
+template <class E>
+attn_status_t combine_impl(const float* o_part, const float* lse_part, void* o, float* lse, int B, int Hq,
+                           int num_splits, int d, attn_stream_t stream) {
+    if (!aligned16(o_part) || !aligned16(lse_part) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_INVALID_ARG;
+    if (B < 1 || Hq < 1 || num_splits < 1) return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    const long long blocks = static_cast<long long>(B) * Hq;
+    const size_t smem = static_cast<size_t>(num_splits) * sizeof(float);
+    if (blocks > 0x7fffffffLL || smem > 48 * 1024) return ATTN_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    auto* ob = static_cast<typename E::T*>(o);
+    if (d == 128)
+        combine_kernel<128, E><<<static_cast<unsigned>(blocks), 128, smem, st>>>(o_part, lse_part, ob, lse, num_splits);
+    else
+        combine_kernel<64, E><<<static_cast<unsigned>(blocks), 64, smem, st>>>(o_part, lse_part, ob, lse, num_splits);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 }  // namespace
@@ -144,56 +197,39 @@ const char* attn_status_string(attn_status_t s) {
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                        int N, int d, int causal, float scale, attn_stream_t stream) {
-    return fwd_impl<false>(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream);
+    return fwd_impl<false, ElemBf16>(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream);
 }
 
 attn_status_t attn_fwd_f32(const void* q, const void* k, const void* v, float* o, float* lse, int B, int Hq,
                            int Hkv, int N, int d, int causal, float scale, attn_stream_t stream) {
-    return fwd_impl<true>(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream);
+    return fwd_impl<true, ElemBf16>(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream);
+}
+
+attn_status_t attn_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                           int N, int d, int causal, float scale, attn_stream_t stream) {
+    return fwd_impl<false, ElemF16>(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream);
 }
 
 attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
                                   int B, int Hq, int Hkv, int L, int d, int num_splits, float scale,
                                   attn_stream_t stream) {
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part) || !aligned16(lse_part))
-        return ATTN_ERR_INVALID_ARG;
-    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0 || num_splits < 1 || num_splits > L ||
-        !scale_ok(scale))
-        return ATTN_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-    if (B > 65535 || num_splits > 0x7fffffff / 2) return ATTN_ERR_INVALID_ARG;
-    const int per = (L + num_splits - 1) / num_splits;
-    const int chunk = (per + 127) / 128 * 128;  // whole 128-key tiles
-    CUtensorMap tk, tv;
-    if (!make_map(&tk, k, d, L, B * Hkv, 128) || !make_map(&tv, v, d, L, B * Hkv, 128)) return ATTN_ERR_CUDA;
-    DecodeParams p;
-    p.q = static_cast<const __nv_bfloat16*>(q);
-    p.o_part = o_part;
-    p.lse_part = lse_part;
-    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.S = num_splits; p.chunk = chunk;
-    p.G = Hq / Hkv;
-    p.groups = (p.G + 127) / 128;  // query heads of a KV head, 128 rows per block
-    if (static_cast<long long>(Hkv) * p.groups > 65535) return ATTN_ERR_INVALID_ARG;
-    p.scale_log2 = scale * kLog2e;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    return d == 128 ? launch_decode<128>(tk, tv, p, st) : launch_decode<64>(tk, tv, p, st);
+    return decode_impl<ElemBf16>(q, k, v, o_part, lse_part, B, Hq, Hkv, L, d, num_splits, scale, stream);
+}
+
+attn_status_t attn_decode_splitkv_f16(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
+                                      int B, int Hq, int Hkv, int L, int d, int num_splits, float scale,
+                                      attn_stream_t stream) {
+    return decode_impl<ElemF16>(q, k, v, o_part, lse_part, B, Hq, Hkv, L, d, num_splits, scale, stream);
 }
 
 attn_status_t attn_combine(const float* o_part, const float* lse_part, void* o, float* lse, int B, int Hq,
                            int num_splits, int d, attn_stream_t stream) {
-    if (!aligned16(o_part) || !aligned16(lse_part) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_INVALID_ARG;
-    if (B < 1 || Hq < 1 || num_splits < 1) return ATTN_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-    const long long blocks = static_cast<long long>(B) * Hq;
-    const size_t smem = static_cast<size_t>(num_splits) * sizeof(float);
-    if (blocks > 0x7fffffffLL || smem > 48 * 1024) return ATTN_ERR_INVALID_ARG;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
-    if (d == 128)
-        combine_kernel<128><<<static_cast<unsigned>(blocks), 128, smem, st>>>(o_part, lse_part, ob, lse, num_splits);
-    else
-        combine_kernel<64><<<static_cast<unsigned>(blocks), 64, smem, st>>>(o_part, lse_part, ob, lse, num_splits);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    return combine_impl<ElemBf16>(o_part, lse_part, o, lse, B, Hq, num_splits, d, stream);
+}
+
+attn_status_t attn_combine_f16(const float* o_part, const float* lse_part, void* o, float* lse, int B, int Hq,
+                               int num_splits, int d, attn_stream_t stream) {
+    return combine_impl<ElemF16>(o_part, lse_part, o, lse, B, Hq, num_splits, d, stream);
 }
 
 attn_status_t attn_merge(float* o_acc, float* lse_acc, const float* o_blk, const float* lse_blk, void* out,

@@ -54,7 +54,7 @@
 namespace eab {
 
 struct FwdParams {
-    void* o;           // [B, Hq, N, D]: bf16, or fp32 for the F32OUT kernels
+    void* o;           // [B, Hq, N, D]: the input type (bf16 / fp16), or fp32 for F32OUT
     float* lse;        // [B, Hq, N]
     int B, Hq, Hkv, N;
     int n_qblocks;     // ceil(N / 256)
@@ -126,7 +126,7 @@ __device__ __forceinline__ float max64(const float (&v)[64]) {
     return max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
-template <int D, bool CAUSAL, bool F32OUT>
+template <int D, bool CAUSAL, bool F32OUT, class E>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -254,8 +254,8 @@ __global__ void __launch_bounds__(384, 1)
         // ---------------------------------------------------- MMA issuers ---
         const int t = warp - 8;
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = make_idesc_bf16(BM, BN, 0, 0);
-            constexpr uint32_t idesc_pv = make_idesc_bf16(BM, D, 0, 1);
+            constexpr uint32_t idesc_qk = make_idesc(BM, BN, 0, 0, E::fmt);
+            constexpr uint32_t idesc_pv = make_idesc(BM, D, 0, 1, E::fmt);
             const uint32_t s_tmem = tmem + t * 256, o_tmem = s_tmem + 128;
             const uint32_t q_addr = smem_addr(sQ + t * C::Q_TILE_BYTES), kv_addr = smem_addr(sKV);
             bool ok = true;
@@ -432,7 +432,7 @@ __global__ void __launch_bounds__(384, 1)
                                                c2x2, negm2);
                         const float2 pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
                         rsum[i & 3] = fadd2(rsum[i & 3], pp);
-                        pk[i] = pack_bf16x2(pp.x, pp.y);
+                        pk[i] = E::pack2(pp.x, pp.y);
                     }
                     tmem_st32(s_addr + half * 32, pk);
                     if (half == 0) {
@@ -498,7 +498,7 @@ __global__ void __launch_bounds__(384, 1)
                     __syncwarp();
                 }
             } else {
-            __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(p.o);
+            auto* ob = static_cast<typename E::T*>(p.o);
 #pragma unroll
             for (int half = 0; half < D / 64; ++half) {
                 // this lane's row, columns [64*half, 64*half + 64): 128 bytes as 8
@@ -518,10 +518,10 @@ __global__ void __launch_bounds__(384, 1)
                     for (int i = 0; i < 4; ++i) {
                         const int chunk = c2 * 4 + i;
                         const uint4 v4 = make_uint4(
-                            pack_bf16x2(__uint_as_float(r3[8 * i + 0]) * inv_l, __uint_as_float(r3[8 * i + 1]) * inv_l),
-                            pack_bf16x2(__uint_as_float(r3[8 * i + 2]) * inv_l, __uint_as_float(r3[8 * i + 3]) * inv_l),
-                            pack_bf16x2(__uint_as_float(r3[8 * i + 4]) * inv_l, __uint_as_float(r3[8 * i + 5]) * inv_l),
-                            pack_bf16x2(__uint_as_float(r3[8 * i + 6]) * inv_l, __uint_as_float(r3[8 * i + 7]) * inv_l));
+                            E::pack2(__uint_as_float(r3[8 * i + 0]) * inv_l, __uint_as_float(r3[8 * i + 1]) * inv_l),
+                            E::pack2(__uint_as_float(r3[8 * i + 2]) * inv_l, __uint_as_float(r3[8 * i + 3]) * inv_l),
+                            E::pack2(__uint_as_float(r3[8 * i + 4]) * inv_l, __uint_as_float(r3[8 * i + 5]) * inv_l),
+                            E::pack2(__uint_as_float(r3[8 * i + 6]) * inv_l, __uint_as_float(r3[8 * i + 7]) * inv_l));
                         *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = v4;
                     }
                 }

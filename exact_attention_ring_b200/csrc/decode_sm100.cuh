@@ -31,7 +31,7 @@
 namespace eab {
 
 struct DecodeParams {
-    const __nv_bfloat16* q;  // [B, Hq, D]
+    const void* q;           // [B, Hq, D], the input type
     float* o_part;           // [B, Hq, S, D]
     float* lse_part;         // [B, Hq, S]
     int B, Hq, Hkv, L, S, chunk;  // chunk: keys per split, a multiple of 128
@@ -67,7 +67,7 @@ __device__ __forceinline__ bool dec_load_kind(int i, int n, int* j) {
     return true;
 }
 
-template <int D>
+template <int D, class E>
 __global__ void __launch_bounds__(224, 1)
     decode_splitkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const DecodeParams p) {
@@ -161,8 +161,8 @@ __global__ void __launch_bounds__(224, 1)
     } else if (warp == 4) {
         // ---------------------------------------------------- MMA issuer ----
         if (lane == 0 && nt > 0) {
-            constexpr uint32_t idesc_qk = make_idesc_bf16(BM, BN, 0, 0);
-            constexpr uint32_t idesc_pv = make_idesc_bf16(BM, D, 0, 1);
+            constexpr uint32_t idesc_qk = make_idesc(BM, BN, 0, 0, E::fmt);
+            constexpr uint32_t idesc_pv = make_idesc(BM, D, 0, 1, E::fmt);
             const uint32_t o_tmem = tmem + 256;
             const uint32_t q_addr = smem_addr(sQ), kv_addr = smem_addr(sKV);
             bool ok = mbar_wait(q_ready, 0, abort_flag);
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
             for (int c = 0; c < D / 8; ++c) {
                 uint4 v4 = make_uint4(0u, 0u, 0u, 0u);
-                if (real) v4 = *reinterpret_cast<const uint4*>(p.q + out_row * D + c * 8);
+                if (real) v4 = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.q) + out_row * D + c * 8);
                 *reinterpret_cast<uint4*>(sQ + (c >> 3) * (BM * 128) + row * 128 + (((c & 7) ^ (row & 7)) << 4)) = v4;
             }
             fence_proxy_async_smem();
@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(224, 1)
                         const float2 y = ffma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2x2, negm2);
                         const float2 pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
                         rsum[i & 3] = fadd2(rsum[i & 3], pp);
-                        pk[i] = pack_bf16x2(pp.x, pp.y);
+                        pk[i] = E::pack2(pp.x, pp.y);
                     }
                     tmem_st32(s_addr + h * 32, pk);
                 }
@@ -339,10 +339,10 @@ __global__ void __launch_bounds__(224, 1)
 // ------------------------------------------------------------- combine ------
 // One block per (b, h), D threads: M = max_s lse_s, w_s = exp(lse_s - M),
 // O = sum_s w_s O_s / sum_s w_s, LSE = M + ln(sum_s w_s).
-template <int D>
+template <int D, class E>
 __global__ void __launch_bounds__(D)
     combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
-                   __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int S) {
+                   typename E::T* __restrict__ o, float* __restrict__ lse, int S) {
     extern __shared__ float w_s[];  // S weights
     __shared__ float red[D / 32];
     __shared__ float bcast;
@@ -386,7 +386,7 @@ __global__ void __launch_bounds__(D)
     float acc = 0.f;
     for (int s = 0; s < S; ++s) acc = fmaf(w_s[s], op[static_cast<size_t>(s) * D], acc);
     const bool none = !(wsum > 0.f);
-    o[static_cast<size_t>(bh) * D + t] = __float2bfloat16_rn(none ? 0.f : acc / wsum);
+    o[static_cast<size_t>(bh) * D + t] = E::from_float(none ? 0.f : acc / wsum);
     if (t == 0) lse[bh] = none ? -INFINITY : M + logf(wsum);
 }
 

@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace eab {
 
@@ -183,12 +184,12 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         : "memory");
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and an fp32 accumulator.
-// Fields: c_format [4,6) = 1 (F32); a_format [7,10) = 1 (BF16); b_format
-// [10,13) = 1 (BF16); a_major bit 15; b_major bit 16 (0 = K-major, 1 = MN-major);
-// N >> 3 in [17,23); M >> 4 in [24,29).
-__host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn_major) << 15) | (uint32_t(b_mn_major) << 16) |
+// Instruction descriptor for kind::f16 with 16-bit A/B of one type (fmt 0 =
+// F16, 1 = BF16; one MMA never mixes them) and an fp32 accumulator. Fields:
+// c_format [4,6) = 1 (F32); a_format [7,10); b_format [10,13); a_major bit 15;
+// b_major bit 16 (0 = K-major, 1 = MN-major); N >> 3 in [17,23); M >> 4 in [24,29).
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N, int a_mn_major, int b_mn_major, uint32_t fmt) {
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | (uint32_t(a_mn_major) << 15) | (uint32_t(b_mn_major) << 16) |
            (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
@@ -298,6 +299,26 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
 }
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// The 16-bit input types: the MMA format code, and rounding (to nearest even)
+// of results into them.
+struct ElemBf16 {
+    using T = __nv_bfloat16;
+    static constexpr uint32_t fmt = 1;
+    static __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
+    static __device__ __forceinline__ T from_float(float x) { return __float2bfloat16_rn(x); }
+};
+struct ElemF16 {
+    using T = __half;
+    static constexpr uint32_t fmt = 0;
+    static __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_f16x2(lo, hi); }
+    static __device__ __forceinline__ T from_float(float x) { return __float2half_rn(x); }
+};
 
 // Warpgroup register reallocation (every warp of the warpgroup executes it).
 template <uint32_t N>

@@ -142,6 +142,24 @@ attn_status_t attn_merge(float* o_acc, float* lse_acc, const float* o_blk, const
                          void* out, long long rows, int d, int init, attn_stream_t stream);
 
 /*
+ * attn_fwd_f16, attn_decode_splitkv_f16, attn_combine_f16 — the same three calls
+ * for IEEE fp16 inputs (the pages list FP16 beside BF16 among the supported
+ * dtypes: "1-Flash-Attention.md", "使用注意事项"). Arguments, layouts, checks and
+ * errors as for the bf16 calls; every 16-bit buffer (q, k, v, o) holds fp16
+ * bit patterns, P is rounded to fp16 for the P V product, and o is written as
+ * fp16 (round to nearest even). lse and the split partials stay fp32.
+ */
+attn_status_t attn_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                           attn_stream_t stream);
+attn_status_t attn_decode_splitkv_f16(const void* q, const void* k, const void* v,
+                                      float* o_part, float* lse_part,
+                                      int B, int Hq, int Hkv, int L, int d, int num_splits,
+                                      float scale, attn_stream_t stream);
+attn_status_t attn_combine_f16(const float* o_part, const float* lse_part, void* o, float* lse,
+                               int B, int Hq, int num_splits, int d, attn_stream_t stream);
+
+/*
  * attn_decode_default_splits — the split count attn_decode_splitkv is tuned for
  * on a 148-SM B200: it maximises the busy fraction of the waves of (batch,
  * kv-head, split) blocks times the fraction of each block's time spent

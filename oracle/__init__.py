@@ -18,7 +18,7 @@ import torch
 from .build import build_oracle, library_path
 
 _lib = None
-_DT = {torch.float64: 0, torch.bfloat16: 1, torch.float32: 2}
+_DT = {torch.float64: 0, torch.bfloat16: 1, torch.float32: 2, torch.float16: 3}
 
 
 def _load(plant: int = 0):
@@ -44,6 +44,8 @@ def _bind(lib):
     lib.oracle_combine.argtypes = [P, P, I, I, I, I, P, P]
     lib.oracle_combine.restype = I
     lib.oracle_hardware_threads.restype = I
+    lib.oracle_widen.argtypes = [I, P, L, P]
+    lib.oracle_widen.restype = I
     return lib
 
 
@@ -150,3 +152,15 @@ def decode(q, k, v, scale: float, rows=None, nthreads: int = 0):
     if rows is None:
         return o.view(B, Hq, d), lse.view(B, Hq)
     return o, lse
+
+
+def widen(x):
+    """The oracle's own widening of an input tensor (any of its input types) to
+    float64, element by element (test hook for the format conversions)."""
+    x = x.contiguous()
+    n = x.numel()
+    lib = _load()
+    out = torch.empty(n, dtype=torch.float64)
+    rc = lib.oracle_widen(_DT[x.dtype], _ptr(x), n, _ptr(out))
+    _check(rc, "widen")
+    return out.view(x.shape)

@@ -43,13 +43,29 @@ namespace {
 
 constexpr int kPlant = ORACLE_PLANT;
 
-enum InType { IN_F64 = 0, IN_BF16 = 1, IN_F32 = 2 };
+enum InType { IN_F64 = 0, IN_BF16 = 1, IN_F32 = 2, IN_F16 = 3 };
+
+// IEEE 754 binary16 -> double from the format's definition: sign bit, 5
+// exponent bits with bias 15, 10 fraction bits; exponent 0 holds zero and the
+// subnormals (fraction * 2^-24), exponent 31 the infinities and NaN.
+inline double half_to_double(uint16_t h) {
+    const int sign = (h >> 15) & 1, e = (h >> 10) & 31, f = h & 1023;
+    double mag;
+    if (e == 0)
+        mag = std::ldexp(static_cast<double>(f), -24);
+    else if (e == 31)
+        mag = f ? std::numeric_limits<double>::quiet_NaN() : std::numeric_limits<double>::infinity();
+    else
+        mag = std::ldexp(1.0 + f / 1024.0, e - 15);
+    return sign ? -mag : mag;
+}
 
 // bf16 -> double: a bf16 value is the top 16 bits of an IEEE float32.
 inline double load_elem(int dtype, const void* base, int64_t idx) {
     switch (dtype) {
         case IN_F64: return static_cast<const double*>(base)[idx];
         case IN_F32: return static_cast<const float*>(base)[idx];
+        case IN_F16: return half_to_double(static_cast<const uint16_t*>(base)[idx]);
         default: {
             uint32_t bits = static_cast<uint32_t>(static_cast<const uint16_t*>(base)[idx]) << 16;
             float f;
@@ -261,6 +277,14 @@ int oracle_decode_partials(int dtype, const void* q, const void* k, const void* 
 
 // Logsumexp-weighted merge: M = max_s lse_s, w_s = exp(lse_s - M),
 // O = sum_s w_s O_s / sum_s w_s, LSE = M + ln sum_s w_s.
+// Widens n elements of one of the input types to double (exposes load_elem to
+// the tests that pin the format conversions).
+int oracle_widen(int dtype, const void* x, int64_t n, double* out) {
+    if (x == nullptr || out == nullptr || n < 0 || dtype < IN_F64 || dtype > IN_F16) return 1;
+    for (int64_t i = 0; i < n; ++i) out[i] = load_elem(dtype, x, i);
+    return 0;
+}
+
 int oracle_combine(const double* o_part, const double* lse_part, int B, int Hq, int num_splits,
                    int d, double* o, double* lse) {
     if (B < 1 || Hq < 1 || num_splits < 1 || d < 1) return 1;

@@ -23,35 +23,37 @@ from dataclasses import dataclass, field
 import torch
 
 
-def _randn_bf16(gen: torch.Generator, shape) -> torch.Tensor:
-    return torch.randn(*shape, generator=gen, dtype=torch.float32).to(torch.bfloat16)
+def _randn_bf16(gen: torch.Generator, shape, dtype=torch.bfloat16) -> torch.Tensor:
+    # N(0,1) drawn in fp32, then rounded (RNE) to the input type
+    return torch.randn(*shape, generator=gen, dtype=torch.float32).to(dtype)
 
 
-def make_qkv(seed: int, B: int, Hq: int, Hkv: int, N: int, d: int, q_mult: float = 1.0):
-    """Prefill inputs: (q, k, v) as contiguous bf16 CPU tensors."""
+def make_qkv(seed: int, B: int, Hq: int, Hkv: int, N: int, d: int, q_mult: float = 1.0,
+             dtype=torch.bfloat16):
+    """Prefill inputs: (q, k, v) as contiguous CPU tensors (bf16, or fp16)."""
     gen = torch.Generator().manual_seed(seed)
-    q = _randn_bf16(gen, (B, Hq, N, d))
-    k = _randn_bf16(gen, (B, Hkv, N, d))
-    v = _randn_bf16(gen, (B, Hkv, N, d))
+    q = _randn_bf16(gen, (B, Hq, N, d), dtype)
+    k = _randn_bf16(gen, (B, Hkv, N, d), dtype)
+    v = _randn_bf16(gen, (B, Hkv, N, d), dtype)
     if q_mult != 1.0:
-        assert math.log2(q_mult).is_integer(), "q_mult must be a power of two (exact in bf16)"
-        q = (q.float() * q_mult).to(torch.bfloat16)
+        assert math.log2(q_mult).is_integer(), "q_mult must be a power of two (exact in bf16 and fp16)"
+        q = (q.float() * q_mult).to(dtype)
     return q.contiguous(), k.contiguous(), v.contiguous()
 
 
-def make_decode(seed: int, B: int, Hq: int, Hkv: int, L: int, d: int, pin: bool = False):
-    """Single-query decode inputs: q [B,Hq,d], k/v [B,Hkv,L,d], bf16 CPU tensors.
+def make_decode(seed: int, B: int, Hq: int, Hkv: int, L: int, d: int, pin: bool = False, dtype=torch.bfloat16):
+    """Single-query decode inputs: q [B,Hq,d], k/v [B,Hkv,L,d], CPU tensors (bf16, or fp16).
 
     Drawn in the order q, then k one batch entry at a time, then v likewise,
     so that a large cache never needs a full float32 copy on the host.
     """
     gen = torch.Generator().manual_seed(seed)
-    q = _randn_bf16(gen, (B, Hq, d)).contiguous()
-    k = torch.empty(B, Hkv, L, d, dtype=torch.bfloat16, pin_memory=pin)
-    v = torch.empty(B, Hkv, L, d, dtype=torch.bfloat16, pin_memory=pin)
+    q = _randn_bf16(gen, (B, Hq, d), dtype).contiguous()
+    k = torch.empty(B, Hkv, L, d, dtype=dtype, pin_memory=pin)
+    v = torch.empty(B, Hkv, L, d, dtype=dtype, pin_memory=pin)
     for t in (k, v):
         for b in range(B):
-            t[b] = _randn_bf16(gen, (Hkv, L, d))
+            t[b] = _randn_bf16(gen, (Hkv, L, d), dtype)
     return q, k, v
 
 

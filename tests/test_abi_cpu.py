@@ -57,6 +57,25 @@ def _fwd32(lib, q=16, k=32, v=48, o=64, lse=80, B=1, Hq=2, Hkv=1, N=8, d=64, cau
     return lib.attn_fwd_f32(P(q), P(k), P(v), P(o), P(lse), B, Hq, Hkv, N, d, causal, ctypes.c_float(scale), None)
 
 
+def _fwd16(lib, q=16, k=32, v=48, o=64, lse=80, B=1, Hq=2, Hkv=1, N=8, d=64, causal=0, scale=0.125):
+    P = ctypes.c_void_p
+    lib.attn_fwd_f16.restype = ctypes.c_int
+    return lib.attn_fwd_f16(P(q), P(k), P(v), P(o), P(lse), B, Hq, Hkv, N, d, causal, ctypes.c_float(scale), None)
+
+
+def _dec16(lib, q=16, k=32, v=48, op=64, lp=80, B=1, Hq=4, Hkv=2, L=100, d=128, S=4, scale=0.1):
+    P = ctypes.c_void_p
+    lib.attn_decode_splitkv_f16.restype = ctypes.c_int
+    return lib.attn_decode_splitkv_f16(P(q), P(k), P(v), P(op), P(lp), B, Hq, Hkv, L, d, S, ctypes.c_float(scale),
+                                       None)
+
+
+def _comb16(lib, op=16, lp=32, o=48, lse=64, B=1, Hq=4, S=3, d=64):
+    P = ctypes.c_void_p
+    lib.attn_combine_f16.restype = ctypes.c_int
+    return lib.attn_combine_f16(P(op), P(lp), P(o), P(lse), B, Hq, S, d, None)
+
+
 def _dec(lib, q=16, k=32, v=48, op=64, lp=80, B=1, Hq=4, Hkv=2, L=100, d=128, S=4, scale=0.1):
     P = ctypes.c_void_p
     lib.attn_decode_splitkv.restype = ctypes.c_int
@@ -130,6 +149,25 @@ def test_merge_rejects_invalid(lib, kw):
 @pytest.mark.parametrize("d", [0, 32, 96, 256])
 def test_merge_rejects_unsupported_head_dim(lib, d):
     assert _merge(lib, d=d) == UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw", [dict(q=0), dict(o=24), dict(N=0), dict(Hq=3, Hkv=2), dict(causal=2), dict(scale=0.0)])
+def test_fwd_f16_rejects_invalid(lib, kw):
+    assert _fwd16(lib, **kw) == INVALID
+
+
+@pytest.mark.parametrize("kw", [dict(q=0), dict(lp=8), dict(L=0), dict(S=0), dict(Hq=5, Hkv=2)])
+def test_decode_f16_rejects_invalid(lib, kw):
+    assert _dec16(lib, **kw) == INVALID
+
+
+@pytest.mark.parametrize("kw", [dict(op=0), dict(lse=4), dict(S=0)])
+def test_combine_f16_rejects_invalid(lib, kw):
+    assert _comb16(lib, **kw) == INVALID
+
+
+def test_f16_calls_reject_unsupported_head_dim(lib):
+    assert _fwd16(lib, d=96) == UNSUPPORTED and _dec16(lib, d=80) == UNSUPPORTED and _comb16(lib, d=100) == UNSUPPORTED
 
 
 def test_status_strings(lib):

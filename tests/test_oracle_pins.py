@@ -212,6 +212,28 @@ def pin_bf16_inputs_widen_exactly(plant=0):
     assert torch.equal(ob, od) and torch.equal(lb, ld)
 
 
+def pin_fp16_inputs_widen_exactly(plant=0):
+    """fp16 inputs: the oracle's own binary16 decoding agrees with torch's on all
+    65,536 bit patterns, and fp16 inputs give the same answer as their values
+    passed as float64."""
+    bits = torch.arange(65536, dtype=torch.int32).to(torch.int16).view(torch.float16)
+    w, ref = oracle.widen(bits), bits.to(torch.float64)
+    nan = torch.isnan(ref)
+    assert torch.equal(torch.isnan(w), nan) and torch.equal(w[~nan], ref[~nan])
+    q, k, v = (_rand(s, 1, 2, 9, 8).to(torch.float16) for s in (83, 84, 85))
+    oh, lh = oracle.attention(q, k, v, True, 0.3, plant=plant)
+    od, ld = oracle.attention(q.double(), k.double(), v.double(), True, 0.3, plant=plant)
+    assert torch.equal(oh, od) and torch.equal(lh, ld)
+
+
+def test_bf16_widening_matches_torch():
+    """The oracle's bf16 decoding agrees with torch's on all 65,536 bit patterns."""
+    bits = torch.arange(65536, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    w, ref = oracle.widen(bits), bits.to(torch.float64)
+    nan = torch.isnan(ref)
+    assert torch.equal(torch.isnan(w), nan) and torch.equal(w[~nan], ref[~nan])
+
+
 def pin_row_sampling(plant=0):
     """Computing a subset of rows gives exactly those rows of the full result."""
     q, k, v = _rand(90, 2, 3, 20, 4), _rand(91, 2, 3, 20, 4), _rand(92, 2, 3, 20, 4)
@@ -224,7 +246,7 @@ def pin_row_sampling(plant=0):
 PINS = [pin_probs_are_distributions, pin_constant_v, pin_causal_first_row, pin_single_key,
         pin_two_keys_closed_form, pin_identical_keys, pin_library_sdpa, pin_brute_force_tiny,
         pin_blockwise_equals_direct, pin_invariants, pin_decode_and_combine,
-        pin_bf16_inputs_widen_exactly, pin_row_sampling]
+        pin_bf16_inputs_widen_exactly, pin_fp16_inputs_widen_exactly, pin_row_sampling]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
