@@ -15,10 +15,10 @@
 // heaviest first and dealt to the CTAs in snake order. 384 threads,
 // warp-specialised:
 //   warps 0-3   softmax of query tile 0, one thread per row (TMEM lane), and
-//               its epilogue: O/l to bf16, staged per warp in shared memory
-//               (32 rows x 64 columns at a time, 16-byte chunks XOR-swizzled)
-//               and read back so that every store writes whole 128-byte row
-//               segments;
+//               its epilogue: O/l rounded to the input type (or kept in fp32
+//               for the F32OUT kernels), staged per warp in shared memory
+//               (16-byte chunks XOR-swizzled) and read back so that every
+//               store writes whole 128-byte row segments;
 //   warps 4-7   the same for query tile 1;
 //   warp 8, 9   MMA issuers, one per query tile. A thread that has just issued
 //               tcgen05.mma cannot act on an mbarrier for several hundred cycles,
@@ -34,7 +34,8 @@
 //                             in TMEM (lazy rescale); the two softmax warpgroups
 //                             then take turns for pass 2, which computes
 //                             p = exp2(s*scale*log2e - m) with one FMA, sums l in
-//                             fp32 and writes P_t as bf16 over the S_t columns,
+//                             fp32 and writes P_t in the input type (bf16 or
+//                             fp16, the E template parameter) over the S_t columns,
 //                             announcing each half (64 keys) as it lands;
 //   O_t += P_t V_j            tcgen05.mma with A = P_t from TMEM, B = V_j MN-major,
 //                             the first 64 keys while the softmax still works on
