@@ -52,11 +52,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # it was taken on (sha256 of the kernel file, first 16 hex digits).
 NCU_TRAFFIC = {
     # decode_splitkv_kernel<128>, B1 Hq32 Hkv8 L131072 d128 (the bench's decode workload)
-    "decode": {"bytes_per_launch": 536931840 + 3522304, "source_sha": "47462cbad1d67d1c"},
+    "decode": {"bytes_per_launch": 536948992 + 3485696, "source_sha": "4b6ee8ffded319ea"},
     # attn_fwd_kernel<128,causal / non-causal>, B2 H32 N2048 d128 (the bench's prefill workloads),
     # read + write with cold caches (ncu flushes them before each captured launch)
-    "attn_fwd_causal": {"bytes_per_launch": 148234496 + 16394240, "source_sha": "ed115c8fd1b2acdf"},
-    "attn_fwd_noncausal": {"bytes_per_launch": 259220992 + 27508224, "source_sha": "ed115c8fd1b2acdf"},
+    "attn_fwd_causal": {"bytes_per_launch": 149111296 + 16082944, "source_sha": "30dee28611453093"},
+    "attn_fwd_noncausal": {"bytes_per_launch": 269126144 + 28518144, "source_sha": "30dee28611453093"},
 }
 
 
