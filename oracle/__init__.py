@@ -46,6 +46,8 @@ def _bind(lib):
     lib.oracle_hardware_threads.restype = I
     lib.oracle_widen.argtypes = [I, P, L, P]
     lib.oracle_widen.restype = I
+    lib.oracle_attention_backward.argtypes = [I, P, P, P, P, I, I, I, I, I, I, D, P, P, P, I]
+    lib.oracle_attention_backward.restype = I
     return lib
 
 
@@ -164,3 +166,20 @@ def widen(x):
     rc = lib.oracle_widen(_DT[x.dtype], _ptr(x), n, _ptr(out))
     _check(rc, "widen")
     return out.view(x.shape)
+
+
+def attention_backward(q, k, v, dout, causal: bool, scale: float, nthreads: int = 0):
+    """Gradients of sum(dout * O) for O = softmax(scale Q K^T) V (masked):
+    returns (dq [B,Hq,N,d], dk [B,Hkv,N,d], dv [B,Hkv,N,d]) as float64."""
+    q, k, v, dt = _prep(q, k, v)
+    dout = dout.contiguous()
+    assert dout.dtype == q.dtype and dout.shape == q.shape
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    dq = torch.empty(B, Hq, N, d, dtype=torch.float64)
+    dk = torch.empty(B, Hkv, N, d, dtype=torch.float64)
+    dv = torch.empty(B, Hkv, N, d, dtype=torch.float64)
+    rc = _load().oracle_attention_backward(dt, _ptr(q), _ptr(k), _ptr(v), _ptr(dout), B, Hq, Hkv, N, d,
+                                           int(causal), float(scale), _ptr(dq), _ptr(dk), _ptr(dv), nthreads)
+    _check(rc, "attention_backward")
+    return dq, dk, dv

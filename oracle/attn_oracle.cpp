@@ -277,6 +277,67 @@ int oracle_decode_partials(int dtype, const void* q, const void* k, const void* 
 
 // Logsumexp-weighted merge: M = max_s lse_s, w_s = exp(lse_s - M),
 // O = sum_s w_s O_s / sum_s w_s, LSE = M + ln sum_s w_s.
+// Gradients of the scalar sum(dO * O) with respect to Q, K and V, from the
+// definition (backward pass; the forward's LSE is recomputed, not taken from
+// the GPU): for the visible keys j of row i, with P the softmax of the row,
+//   dP_ij = dO_i . v_j,   Delta_i = sum_j P_ij dP_ij,   dS_ij = P_ij (dP_ij - Delta_i),
+//   dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i,  dV_j = sum_i P_ij dO_i,
+// dK and dV summed over every query head that reads the key/value head.
+// Threads take whole (batch, key/value head) groups, so no sums are shared.
+int oracle_attention_backward(int dtype, const void* q, const void* k, const void* v, const void* dout, int B,
+                              int Hq, int Hkv, int N, int d, int causal, double scale, double* dq, double* dk,
+                              double* dv, int nthreads) {
+    if (!q || !k || !v || !dout || !dq || !dk || !dv || B < 1 || Hq < 1 || Hkv < 1 || N < 1 || d < 1 ||
+        Hq % Hkv != 0)
+        return 1;
+    Problem p{dtype, q, k, v, B, Hq, Hkv, N, N, d, causal, scale};
+    const int G = Hq / Hkv;
+    const int64_t groups = static_cast<int64_t>(B) * Hkv;
+    const int nt = nthreads > 0 ? nthreads : std::max(1u, std::thread::hardware_concurrency());
+    auto work = [&](int tid) {
+        std::vector<double> s, dp;
+        for (int64_t gidx = tid; gidx < groups; gidx += nt) {
+            const int64_t b = gidx / Hkv, hk = gidx % Hkv;
+            const int64_t kvoff = (b * Hkv + hk) * static_cast<int64_t>(N) * d;
+            for (int64_t e = 0; e < static_cast<int64_t>(N) * d; ++e) dk[kvoff + e] = dv[kvoff + e] = 0.0;
+            for (int64_t h = hk * G; h < (hk + 1) * G; ++h) {
+                for (int64_t i = 0; i < N; ++i) {
+                    const int64_t qoff = ((b * Hq + h) * N + i) * d;
+                    scores(p, b, h, i, s);
+                    const int64_t J = static_cast<int64_t>(s.size());
+                    double m = -std::numeric_limits<double>::infinity();
+                    for (double x : s) m = std::max(m, x);
+                    double l = 0.0;
+                    for (int64_t j = 0; j < J; ++j) { s[j] = std::exp(s[j] - m); l += s[j]; }
+                    for (int64_t j = 0; j < J; ++j) s[j] /= l;  // P_ij
+                    dp.assign(J, 0.0);
+                    double delta = 0.0;
+                    for (int64_t j = 0; j < J; ++j) {
+                        double acc = 0.0;
+                        for (int t = 0; t < d; ++t)
+                            acc += load_elem(dtype, dout, qoff + t) * load_elem(dtype, v, kvoff + j * d + t);
+                        dp[j] = acc;
+                        delta += s[j] * acc;
+                    }
+                    for (int t = 0; t < d; ++t) dq[qoff + t] = 0.0;
+                    for (int64_t j = 0; j < J; ++j) {
+                        const double ds = s[j] * (dp[j] - delta);
+                        for (int t = 0; t < d; ++t) {
+                            dq[qoff + t] += scale * ds * load_elem(dtype, k, kvoff + j * d + t);
+                            dk[kvoff + j * d + t] += scale * ds * load_elem(dtype, q, qoff + t);
+                            dv[kvoff + j * d + t] += s[j] * load_elem(dtype, dout, qoff + t);
+                        }
+                    }
+                }
+            }
+        }
+    };
+    std::vector<std::thread> pool;
+    for (int t = 0; t < nt; ++t) pool.emplace_back(work, t);
+    for (auto& th : pool) th.join();
+    return 0;
+}
+
 // Widens n elements of one of the input types to double (exposes load_elem to
 // the tests that pin the format conversions).
 int oracle_widen(int dtype, const void* x, int64_t n, double* out) {

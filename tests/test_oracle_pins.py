@@ -249,6 +249,44 @@ PINS = [pin_probs_are_distributions, pin_constant_v, pin_causal_first_row, pin_s
         pin_bf16_inputs_widen_exactly, pin_fp16_inputs_widen_exactly, pin_row_sampling]
 
 
+def test_backward_matches_autograd():
+    """The backward pass against torch's float64 autograd of its SDPA (causal
+    and not, grouped heads)."""
+    g = torch.Generator().manual_seed(120)
+    B, Hq, Hkv, N, d = 2, 4, 2, 9, 6
+    for causal in (False, True):
+        q = torch.randn(B, Hq, N, d, generator=g, dtype=torch.float64, requires_grad=True)
+        k = torch.randn(B, Hkv, N, d, generator=g, dtype=torch.float64, requires_grad=True)
+        v = torch.randn(B, Hkv, N, d, generator=g, dtype=torch.float64, requires_grad=True)
+        do = torch.randn(B, Hq, N, d, generator=g, dtype=torch.float64)
+        o = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=causal, scale=0.35, enable_gqa=True)
+        o.backward(do)
+        dq, dk, dv = oracle.attention_backward(q.detach(), k.detach(), v.detach(), do, causal, 0.35)
+        for mine, ref in ((dq, q.grad), (dk, k.grad), (dv, v.grad)):
+            assert torch.allclose(mine, ref, atol=1e-12, rtol=0)
+
+
+def test_backward_matches_finite_differences():
+    """Central differences of sum(dO * O) through the oracle's own forward pass."""
+    g = torch.Generator().manual_seed(121)
+    B, Hq, Hkv, N, d, sc = 1, 2, 1, 5, 3, 0.6
+    q, k, v, do = (torch.randn(*sh, generator=g, dtype=torch.float64)
+                   for sh in ((B, Hq, N, d), (B, Hkv, N, d), (B, Hkv, N, d), (B, Hq, N, d)))
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, True, sc)
+    eps = 1e-6
+
+    def loss(qq, kk, vv):
+        return float((oracle.attention(qq, kk, vv, True, sc)[0] * do).sum())
+
+    for t, grad, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        for idx in range(t.numel()):
+            plus, minus = [q.clone(), k.clone(), v.clone()], [q.clone(), k.clone(), v.clone()]
+            plus[which].view(-1)[idx] += eps
+            minus[which].view(-1)[idx] -= eps
+            fd = (loss(*plus) - loss(*minus)) / (2 * eps)
+            assert abs(fd - grad.view(-1)[idx].item()) < 1e-6
+
+
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
 def test_pin(pin):
     pin()
