@@ -13,6 +13,7 @@ place of pointers; ``stream`` defaults to torch's current stream):
     attn_decode_splitkv(q, k, v, o_part, lse_part, num_splits, scale)
     attn_combine(o_part, lse_part, o, lse)
     attn_merge(o_acc, lse_acc, o_blk, lse_blk, out=None, init=False)
+    attn_bwd(q, k, v, o, lse, dout, delta, dq, dk, dv, causal, scale)   (gradients)
 Ring attention (context parallelism, ``ring.py``): each rank attends its query
 shard to every key/value shard as the shards travel around the ring of ranks,
 merging with attn_merge:
@@ -20,10 +21,13 @@ merging with attn_merge:
 Convenience wrappers that allocate the outputs with torch:
     attention(q, k, v, causal=False, scale=None) -> (o, lse)
     decode(q, k, v, scale=None, num_splits=None) -> (o, lse)
+    attention_backward(q, k, v, o, lse, dout, causal=False, scale=None) -> (dq, dk, dv)
 """
 from ._binding import (  # noqa: F401
     AttnError,
     attention,
+    attention_backward,
+    attn_bwd,
     attn_combine,
     attn_combine_f16,
     attn_decode_default_splits,

@@ -56,6 +56,8 @@ def _load():
     lib.attn_decode_noalloc.restype = I
     lib.attn_merge.argtypes = [P, P, P, P, P, ctypes.c_longlong, I, I, P]
     lib.attn_merge.restype = I
+    lib.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.attn_bwd.restype = I
     return lib
 
 
@@ -128,6 +130,24 @@ def attn_fwd_f32(q, k, v, o, lse, causal: bool, scale: float, stream=None):
         raise ValueError("attn_fwd_f32: inconsistent shapes")
     _check(_lib.attn_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, int(bool(causal)),
                              float(scale), _stream(stream)), "attn_fwd_f32")
+
+
+def attn_bwd(q, k, v, o, lse, dout, delta, dq, dk, dv, causal: bool, scale: float, stream=None):
+    """Gradients of attention: q, o, dout, dq [B,Hq,N,d] and k, v, dk, dv [B,Hkv,N,d]
+    bf16; lse (from attn_fwd) and the workspace delta [B,Hq,N] fp32."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, torch.bfloat16, n)
+    _need(lse, torch.float32, "lse")
+    _need(delta, torch.float32, "delta")
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if (k.shape != (B, Hkv, N, d) or v.shape != k.shape or dk.shape != k.shape or dv.shape != k.shape
+            or o.shape != q.shape or dout.shape != q.shape or dq.shape != q.shape
+            or lse.shape != (B, Hq, N) or delta.shape != (B, Hq, N)):
+        raise ValueError("attn_bwd: inconsistent shapes")
+    _check(_lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(delta), _ptr(dq),
+                         _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream)),
+           "attn_bwd")
 
 
 def _dec(fn, name, dt, q, k, v, o_part, lse_part, num_splits, scale, stream):
@@ -227,6 +247,17 @@ def attention(q, k, v, causal: bool = False, scale: float | None = None, stream=
     lse = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)
     (attn_fwd_f16 if q.dtype == torch.float16 else attn_fwd)(q, k, v, o, lse, causal, scale, stream)
     return o, lse
+
+
+def attention_backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None, stream=None):
+    """Allocates dq, dk, dv (and the Delta workspace) and runs attn_bwd on the
+    forward's (o, lse). Returns (dq, dk, dv) in bf16."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    delta = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)
+    attn_bwd(q, k, v, o, lse, dout, delta, dq, dk, dv, causal, scale, stream)
+    return dq, dk, dv
 
 
 def decode(q, k, v, scale: float | None = None, num_splits: int | None = None, stream=None):

@@ -15,6 +15,7 @@
 
 #include "../../include/attn.h"
 #include "attn_fwd_sm100.cuh"
+#include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "merge_sm100.cuh"
 
@@ -129,6 +130,29 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
         return causal ? launch_fwd<128, true, F32OUT, E>(tq, tk, tv, p, st)
                       : launch_fwd<128, false, F32OUT, E>(tq, tk, tv, p, st);
     return causal ? launch_fwd<64, true, F32OUT, E>(tq, tk, tv, p, st) : launch_fwd<64, false, F32OUT, E>(tq, tk, tv, p, st);
+}
+
+template <int D, bool CAUSAL, bool DKDV>
+attn_status_t launch_bwd_tile(const CUtensorMap& fa, const CUtensorMap& fb, const CUtensorMap& sa,
+                              const CUtensorMap& sb, const BwdParams& p, cudaStream_t stream) {
+    using C = BwdCfg<D>;
+    auto kern = bwd_tile_kernel<D, CAUSAL, DKDV>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    const dim3 grid((p.N + C::BT - 1) / C::BT, p.B * (DKDV ? p.Hkv : p.Hq));
+    kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(fa, fb, sa, sb, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, bool CAUSAL>
+attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+    const long long rows = static_cast<long long>(p.B) * p.Hq * p.N;
+    bwd_delta_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p, rows);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    attn_status_t st = launch_bwd_tile<D, CAUSAL, true>(tk, tv, tq, tdo, p, stream);
+    if (st != ATTN_OK) return st;
+    return launch_bwd_tile<D, CAUSAL, false>(tq, tdo, tk, tv, p, stream);
 }
 
 template <class E>
@@ -247,6 +271,37 @@ attn_status_t attn_merge(float* o_acc, float* lse_acc, const float* o_blk, const
     else
         merge_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(o_acc, lse_acc, o_blk, lse_blk, outb, rows, init);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dout, float* delta, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
+                       int d, int causal, float scale, attn_stream_t stream) {
+    const void* ptrs[] = {q, k, v, o, lse, dout, delta, dq, dk, dv};
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || (causal != 0 && causal != 1) || !scale_ok(scale))
+        return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (static_cast<long long>(B) * Hq > 65535LL) return ATTN_ERR_INVALID_ARG;
+    if ((static_cast<long long>(B) * Hq * N + 7) / 8 > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    CUtensorMap tq, tk, tv, tdo;
+    if (!make_map<ElemBf16>(&tq, q, d, N, B * Hq, 128) || !make_map<ElemBf16>(&tk, k, d, N, B * Hkv, 128) ||
+        !make_map<ElemBf16>(&tv, v, d, N, B * Hkv, 128) || !make_map<ElemBf16>(&tdo, dout, d, N, B * Hq, 128))
+        return ATTN_ERR_CUDA;
+    BwdParams p;
+    p.o = static_cast<const __nv_bfloat16*>(o);
+    p.dout = static_cast<const __nv_bfloat16*>(dout);
+    p.lse = lse;
+    p.delta = delta;
+    p.dq = static_cast<__nv_bfloat16*>(dq);
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N;
+    p.scale = scale;
+    p.scale_log2 = scale * kLog2e;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 128) return causal ? launch_bwd<128, true>(tq, tk, tv, tdo, p, st) : launch_bwd<128, false>(tq, tk, tv, tdo, p, st);
+    return causal ? launch_bwd<64, true>(tq, tk, tv, tdo, p, st) : launch_bwd<64, false>(tq, tk, tv, tdo, p, st);
 }
 
 int attn_decode_default_splits(int B, int Hq, int Hkv, int L) {

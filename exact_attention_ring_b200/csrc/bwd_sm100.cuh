@@ -1,0 +1,355 @@
+// Backward pass on sm_100a: dQ, dK, dV of exact attention from the forward's
+// O and LSE, recomputing P tile by tile.
+//
+// The forward pass keeps only O and the per-row log-sum-exp, so P is rebuilt
+// from S = scale Q K^T and the LSE (FlashAttention V2 page, opening paragraph:
+// tiling plus recomputation, the N x N matrices never written out; Flash
+// Attention notes, "使用注意事项": the backward pass accumulates the softmax
+// terms in fp32). With
+// dP = dO V^T, Delta_i = sum_t dO_it O_it = sum_j P_ij dP_ij and
+// dS = P o (dP - Delta):
+//   dV = P^T dO,   dK = scale dS^T Q,   dQ = scale dS K.
+// Three launches:
+//   bwd_delta_kernel        Delta per row (one warp per row, HBM-bound);
+//   bwd_tile_kernel, DKDV   one 128-key tile of one (batch, KV head) per block:
+//                           for every query head of the group and every query
+//                           tile that sees the keys, S^T = K Q^T and
+//                           dP^T = V dO^T into TMEM, P^T and scale dS^T (bf16)
+//                           written back over them by the element-wise warps
+//                           (one thread per key), then dV += P^T dO and
+//                           dK += scale dS^T Q with A from TMEM;
+//   bwd_tile_kernel, !DKDV  one 128-row query tile of one (batch, query head)
+//                           per block: S = Q K^T and dP = dO V^T per key tile,
+//                           scale dS (bf16) over dP, dQ += scale dS K.
+// 192 threads each: warps 0-3 element-wise work and epilogue (thread = TMEM
+// lane), warp 4 the MMA issuer, warp 5 the TMA producer. The steps of a block
+// run one after another (the MMAs wait for the element-wise pass and back);
+// the next step's S^T / dP^T MMAs are issued after the accumulating MMAs that
+// read P^T / dS^T from the same columns, so the tensor pipe's issue order keeps
+// them intact until read (as in the forward pass). Every wait is bounded.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace eab {
+
+struct BwdParams {
+    const __nv_bfloat16* o;     // [B, Hq, N, D]
+    const __nv_bfloat16* dout;  // [B, Hq, N, D]
+    const float* lse;           // [B, Hq, N]
+    float* delta;               // [B, Hq, N] (written by bwd_delta_kernel)
+    __nv_bfloat16* dq;          // [B, Hq, N, D]
+    __nv_bfloat16* dk;          // [B, Hkv, N, D]
+    __nv_bfloat16* dv;          // [B, Hkv, N, D]
+    int B, Hq, Hkv, N;
+    float scale, scale_log2;
+};
+
+template <int D>
+struct BwdCfg {
+    static constexpr int BT = 128;                 // rows of a query tile / keys of a key tile
+    static constexpr int CHUNKS = D / 64;
+    static constexpr int TILE_BYTES = BT * D * 2;  // one 128 x D bf16 tile
+    static constexpr int NUM_THREADS = 192;
+    // [fixed A, B tiles][2 buffers x 2 streamed tiles][lse/delta 2 x 2 x 128 floats][barriers]
+    static constexpr int SMEM_USED = 1024 + 2 * TILE_BYTES + 4 * TILE_BYTES + 4 * BT * 4 + 16 * 8 + 16;
+    // A block allocates all 512 TMEM columns, so two blocks must never share an
+    // SM (the second would stall in tcgen05.alloc): ask for more than half of
+    // the SM's shared memory.
+    static constexpr int SMEM_BYTES = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+};
+
+// Delta_i = sum_t dO_it O_it, one warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdParams p, long long rows) {
+    const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const int lane = threadIdx.x & 31;
+    constexpr int CPL = D / 32;
+    const __nv_bfloat16* a = p.dout + row * D + lane * CPL;
+    const __nv_bfloat16* b = p.o + row * D + lane * CPL;
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) acc += __bfloat162float(a[i]) * __bfloat162float(b[i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) p.delta[row] = acc;
+}
+
+// Shared skeleton of the two tile kernels. One block owns a fixed pair of
+// tiles (A_fix, B_fix: K and V for dK/dV; Q and dO for dQ) and streams pairs of
+// tiles (S_a, S_b: Q and dO; K and V) through two buffers. Per step:
+//   X = A_fix * S_a^T, Y = B_fix * S_b^T          (both M = 128, N = 128, K = D)
+//   element-wise: P from X and the row/column LSE, G = P o (Y - Delta) * scale
+//   acc1 += P * S_b, acc2 += G * S_a              (dK/dV: A from TMEM)
+// For dQ only acc2 (+= dS K) is kept.
+// TMEM: X [0, 128), Y [128, 256), acc1 [256, 256 + D), acc2 [256 + D, 256 + 2D).
+template <int D, bool CAUSAL, bool DKDV>
+__global__ void __launch_bounds__(192, 1)
+    bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_fa, const __grid_constant__ CUtensorMap tm_fb,
+                    const __grid_constant__ CUtensorMap tm_sa, const __grid_constant__ CUtensorMap tm_sb,
+                    const BwdParams p) {
+    using C = BwdCfg<D>;
+    constexpr int BT = C::BT;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sFA = smem;
+    uint8_t* sFB = sFA + C::TILE_BYTES;
+    uint8_t* sS = sFB + C::TILE_BYTES;  // [2 buffers][S_a, S_b]
+    float* sL = reinterpret_cast<float*>(sS + 4 * C::TILE_BYTES);  // [2 buffers][lse*log2e, delta][128]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sL + 4 * BT);
+    uint64_t* fix_full = bars;       // the fixed tiles loaded
+    uint64_t* st_full = bars + 1;    // [2] streamed tiles of a buffer loaded
+    uint64_t* st_empty = bars + 3;   // [2] streamed tiles of a buffer read by every MMA
+    uint64_t* xy_full = bars + 5;    // X and Y complete
+    uint64_t* pg_full = bars + 6;    // P and G written (4 warp arrivals)
+    uint64_t* l_ready = bars + 7;    // [2] lse/delta of a buffer staged (4 warp arrivals)
+    uint64_t* l_free = bars + 9;     // [2] lse/delta of a buffer read (4 warp arrivals)
+    uint64_t* fin = bars + 11;       // every MMA done
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = p.Hq / p.Hkv;
+    const int n_tiles = (p.N + BT - 1) / BT;
+    // the fixed tile: key tile (dK/dV) or query tile (dQ); under the causal
+    // mask the blocks with the most steps are launched first
+    const int tile = (DKDV || !CAUSAL) ? blockIdx.x : n_tiles - 1 - blockIdx.x;
+    // fixed head (KV head for dK/dV, query head for dQ) and its batch
+    const int b = blockIdx.y / (DKDV ? p.Hkv : p.Hq);
+    const int hfix = blockIdx.y % (DKDV ? p.Hkv : p.Hq);
+    // the streamed steps: dK/dV walks (query head of the group, query tile);
+    // dQ walks key tiles. Causal: query tile >= key tile.
+    const int t_lo = DKDV ? (CAUSAL ? tile : 0) : 0;
+    const int t_hi = DKDV ? n_tiles : (CAUSAL ? tile + 1 : n_tiles);
+    const int per_head = t_hi - t_lo;
+    const int nsteps = DKDV ? G * per_head : per_head;
+
+    if (threadIdx.x == 0) {
+        mbar_init(fix_full, 2 * C::CHUNKS);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&st_full[i], 2 * C::CHUNKS);
+            mbar_init(&st_empty[i], 1);
+            mbar_init(&l_ready[i], 4);
+            mbar_init(&l_free[i], 4);
+        }
+        mbar_init(xy_full, 1);
+        mbar_init(pg_full, 4);
+        mbar_init(fin, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 4) {
+        tmem_alloc(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    // plane (batch * heads + head) and tile row of streamed step s
+    auto step_src = [&](int s, int* plane, int* trow) {
+        if (DKDV) {
+            const int h = hfix * G + s / per_head;
+            *plane = b * p.Hq + h;
+            *trow = (t_lo + s % per_head) * BT;
+        } else {
+            *plane = b * p.Hkv + hfix / G;
+            *trow = (t_lo + s) * BT;
+        }
+    };
+
+    if (warp == 5) {
+        // ------------------------------------------------------ producer ----
+        if (lane == 0 && nsteps > 0) {
+            constexpr uint32_t BOX = BT * 128;
+            const int fplane = DKDV ? b * p.Hkv + hfix : b * p.Hq + hfix;
+#pragma unroll
+            for (int c = 0; c < C::CHUNKS; ++c) {
+                mbar_arrive_expect_tx(fix_full, BOX);
+                tma_load_3d(sFA + c * BOX, &tm_fa, fix_full, c * 64, tile * BT, fplane);
+                mbar_arrive_expect_tx(fix_full, BOX);
+                tma_load_3d(sFB + c * BOX, &tm_fb, fix_full, c * 64, tile * BT, fplane);
+            }
+            int s = 0;
+            for (; s < nsteps; ++s) {
+                const int bu = s & 1;
+                if (s >= 2 && !mbar_wait(&st_empty[bu], ((s >> 1) - 1) & 1, abort_flag)) break;
+                int plane, trow;
+                step_src(s, &plane, &trow);
+                uint8_t* dst = sS + bu * 2 * C::TILE_BYTES;
+#pragma unroll
+                for (int c = 0; c < C::CHUNKS; ++c) {
+                    mbar_arrive_expect_tx(&st_full[bu], BOX);
+                    tma_load_3d(dst + c * BOX, &tm_sa, &st_full[bu], c * 64, trow, plane);
+                    mbar_arrive_expect_tx(&st_full[bu], BOX);
+                    tma_load_3d(dst + C::TILE_BYTES + c * BOX, &tm_sb, &st_full[bu], c * 64, trow, plane);
+                }
+            }
+            // Let every copy in flight land before the CTA can exit.
+            mbar_wait(fix_full, 0, nullptr);
+            for (int i = max(0, s - 2); i < s; ++i) mbar_wait(&st_full[i & 1], (i >> 1) & 1, nullptr);
+        }
+    } else if (warp == 4) {
+        // ---------------------------------------------------- MMA issuer ----
+        if (lane == 0 && nsteps > 0) {
+            constexpr uint32_t idesc_xy = make_idesc(BT, BT, 0, 0, ElemBf16::fmt);  // A, B K-major
+            constexpr uint32_t idesc_acc = make_idesc(BT, D, 0, 1, ElemBf16::fmt);  // B MN-major
+            const uint32_t tX = tmem, tY = tmem + 128, tA1 = tmem + 256, tA2 = tmem + 256 + D;
+            const uint32_t fa = smem_addr(sFA), fb = smem_addr(sFB);
+            bool ok = mbar_wait(fix_full, 0, abort_flag);
+            for (int s = 0; ok && s < nsteps; ++s) {
+                const int bu = s & 1;
+                const uint32_t sa = smem_addr(sS + bu * 2 * C::TILE_BYTES), sb = sa + C::TILE_BYTES;
+                ok = mbar_wait(&st_full[bu], (s >> 1) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                // X = A_fix S_a^T, Y = B_fix S_b^T (after the previous step's
+                // accumulating MMAs have read X and Y: issue order)
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
+                    mma_ss(tX, make_sdesc_sw128(fa + koff, 16, 1024), make_sdesc_sw128(sa + koff, 16, 1024), idesc_xy,
+                           kk > 0 ? 1u : 0u);
+                    mma_ss(tY, make_sdesc_sw128(fb + koff, 16, 1024), make_sdesc_sw128(sb + koff, 16, 1024), idesc_xy,
+                           kk > 0 ? 1u : 0u);
+                }
+                tc_commit(xy_full);
+                ok = mbar_wait_spin(pg_full, s & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                // acc1 += P S_b (dK/dV only: dV += P^T dO), acc2 += G S_a (dK += dS^T Q,
+                // or dQ += dS K); A from TMEM (bf16 packed over X / Y), B MN-major
+#pragma unroll
+                for (int kk = 0; kk < BT / 16; ++kk) {
+                    const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                    if (DKDV)
+                        mma_ts(tA1, tX + kk * 8, make_sdesc_sw128(sb + kk * 16 * 128, BT * 128, 1024), idesc_acc, acc);
+                    mma_ts(tA2, tY + kk * 8, make_sdesc_sw128(sa + kk * 16 * 128, BT * 128, 1024), idesc_acc, acc);
+                }
+                tc_commit(&st_empty[bu]);
+            }
+            tc_commit(fin);
+            mbar_wait(fin, 0, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------- element-wise -----
+        const int row = warp * 32 + lane;  // TMEM lane: key (dK/dV) or query row (dQ)
+        const uint32_t lb = tmem + (uint32_t(warp * 32) << 16);
+        const uint32_t tX = lb, tY = lb + 128, tA1 = lb + 256, tA2 = lb + 256 + D;
+        const float c2 = p.scale_log2;
+        const float LOG2E = 1.4426950408889634f;
+        bool ok = nsteps > 0;
+        // this thread's own row: lse and delta (dQ: fixed query row)
+        float my_l2 = INFINITY, my_delta = 0.f;
+        if (!DKDV) {
+            const int qr = tile * BT + row;
+            if (qr < p.N) {
+                my_l2 = p.lse[static_cast<size_t>(b * p.Hq + hfix) * p.N + qr] * LOG2E;
+                my_delta = p.delta[static_cast<size_t>(b * p.Hq + hfix) * p.N + qr];
+            }
+        }
+        const int fixed_pos = tile * BT + row;  // this thread's key (dK/dV) or query row (dQ)
+        for (int s = 0; ok && s < nsteps; ++s) {
+            const int bu = s & 1;
+            int plane, trow;
+            step_src(s, &plane, &trow);
+            float* lsb = sL + bu * 2 * BT;  // per streamed query row: lse*log2e, then delta
+            if (DKDV) {
+                // stage the streamed query rows' lse and delta (column values)
+                if (s >= 2 && !__all_sync(0xffffffffu, mbar_wait(&l_free[bu], ((s >> 1) - 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                const int qr = trow + row;
+                lsb[row] = qr < p.N ? p.lse[static_cast<size_t>(plane) * p.N + qr] * LOG2E : INFINITY;
+                lsb[BT + row] = qr < p.N ? p.delta[static_cast<size_t>(plane) * p.N + qr] : 0.f;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&l_ready[bu]);
+                if (!__all_sync(0xffffffffu, mbar_wait(&l_ready[bu], (s >> 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(xy_full, s & 1, abort_flag))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t xs[64], ys[64];
+                tmem_ld64(tX + h * 64, xs);
+                tmem_ld64(tY + h * 64, ys);
+                uint32_t pk[32], gk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float pv[2], gv[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int col = h * 64 + 2 * i + e;  // streamed row (dK/dV) or key (dQ) in the tile
+                        const int other = trow + col;
+                        const float l2 = DKDV ? lsb[col] : my_l2;
+                        const float dl = DKDV ? lsb[BT + col] : my_delta;
+                        // visible: query row >= key (causal), and both inside the sequence
+                        const int qpos = DKDV ? other : fixed_pos, kpos = DKDV ? fixed_pos : other;
+                        const bool vis = other < p.N && (!CAUSAL || qpos >= kpos);
+                        const float pr = vis ? ex2_approx(__uint_as_float(xs[2 * i + e]) * c2 - l2) : 0.f;
+                        pv[e] = pr;
+                        gv[e] = pr * (__uint_as_float(ys[2 * i + e]) - dl) * p.scale;
+                    }
+                    pk[i] = pack_bf16x2(pv[0], pv[1]);
+                    gk[i] = pack_bf16x2(gv[0], gv[1]);
+                }
+                if (DKDV) tmem_st32(tX + h * 32, pk);
+                tmem_st32(tY + h * 32, gk);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (DKDV) mbar_arrive(&l_free[bu]);
+                mbar_arrive(pg_full);
+            }
+        }
+        // epilogue: the accumulators (dV, dK; or dQ) to bf16 rows of the output
+        if (ok && __all_sync(0xffffffffu, mbar_wait(fin, 0, abort_flag))) {
+            tc_fence_after();
+            // the TMEM loads are warp-wide; only rows inside the sequence are stored
+            const bool in_seq = fixed_pos < p.N;
+            const size_t out_row =
+                static_cast<size_t>(DKDV ? b * p.Hkv + hfix : b * p.Hq + hfix) * p.N + (in_seq ? fixed_pos : 0);
+#pragma unroll
+            for (int which = 0; which < (DKDV ? 2 : 1); ++which) {
+                __nv_bfloat16* dst = (DKDV ? (which == 0 ? p.dv : p.dk) : p.dq) + out_row * D;
+                const uint32_t src = DKDV ? (which == 0 ? tA1 : tA2) : tA2;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r3[32];
+                    tmem_ld32(src + c * 32, r3);
+                    if (in_seq) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 8)
+                            *reinterpret_cast<uint4*>(dst + c * 32 + i) = make_uint4(
+                                pack_bf16x2(__uint_as_float(r3[i]), __uint_as_float(r3[i + 1])),
+                                pack_bf16x2(__uint_as_float(r3[i + 2]), __uint_as_float(r3[i + 3])),
+                                pack_bf16x2(__uint_as_float(r3[i + 4]), __uint_as_float(r3[i + 5])),
+                                pack_bf16x2(__uint_as_float(r3[i + 6]), __uint_as_float(r3[i + 7])));
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace eab

@@ -4,6 +4,7 @@
     python -m exact_attention_ring_b200.profile_case decode --B 1 --H 32 --Hkv 8 --L 131072 --d 128 --iters 3
     python -m exact_attention_ring_b200.profile_case merge --B 2 --H 32 --N 8192 --d 128 --iters 3
     python -m exact_attention_ring_b200.profile_case ring --B 1 --H 32 --N 16384 --d 128 --world 8 --causal 1
+    python -m exact_attention_ring_b200.profile_case bwd --B 4 --H 32 --N 2048 --d 128 --causal 1 --iters 3
 
 Meant to be wrapped by ncu (one kernel, a few launches, inputs larger than L2
 but a few GB at most). Prints the CUDA-event time of the last launch.
@@ -22,7 +23,7 @@ import seeded_inputs as si  # noqa: E402
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["fwd", "decode", "merge", "ring"])
+    ap.add_argument("kernel", choices=["fwd", "decode", "merge", "ring", "bwd"])
     ap.add_argument("--B", type=int, default=4)
     ap.add_argument("--H", type=int, default=32)
     ap.add_argument("--Hkv", type=int, default=0)
@@ -59,6 +60,19 @@ def main():
             eab.attn_merge(o_acc, lse_acc, o_blk, lse_blk)
             end.record()
         flops = rows * (a.d * (4 + 4 + 4) + 4 * 3)  # bytes for merge
+    elif a.kernel == "bwd":
+        # the three launches of attn_bwd (Delta, dK/dV, dQ) on the forward's O, LSE;
+        # FLOPs counted as the five N x N x d products of the backward pass
+        q, k, v = (t.to(dev) for t in si.make_qkv(1001, a.B, a.H, Hkv, a.N, a.d))
+        do = si.make_dout(1002, a.B, a.H, a.N, a.d).to(dev)
+        o, lse = eab.attention(q, k, v, bool(a.causal), a.d ** -0.5)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        delta = torch.empty_like(lse)
+        for _ in range(a.iters):
+            start.record()
+            eab.attn_bwd(q, k, v, o, lse, do, delta, dq, dk, dv, bool(a.causal), a.d ** -0.5)
+            end.record()
+        flops = 10.0 * a.B * a.H * a.N * a.N * a.d / (2 if a.causal else 1)
     elif a.kernel == "ring":
         # every virtual rank's steps of the ring, one after another on this GPU:
         # the whole ring's attention and merge work (no exchange)
@@ -81,7 +95,7 @@ def main():
     torch.cuda.synchronize()
     assert eab.attn_device_status() == 0
     ms = start.elapsed_time(end)
-    tensor = a.kernel in ("fwd", "ring")
+    tensor = a.kernel in ("fwd", "ring", "bwd")
     unit = "TFLOPS" if tensor else "GB/s"
     val = flops / (ms * 1e-3) / (1e12 if tensor else 1e9)
     print(f"{a.kernel}: {ms:.4f} ms  {val:.1f} {unit}")

@@ -142,6 +142,35 @@ attn_status_t attn_merge(float* o_acc, float* lse_acc, const float* o_blk, const
                          void* out, long long rows, int d, int init, attn_stream_t stream);
 
 /*
+ * attn_bwd — gradients of exact attention with respect to q, k and v, given the
+ * output gradient dout and the forward pass's o and lse (attn_fwd, same inputs).
+ * P is recomputed from q, k and lse instead of being stored (FlashAttention V2
+ * page, opening paragraph: tiling and recomputation; Flash Attention notes,
+ * "使用注意事项": the backward pass keeps the softmax terms in fp32). For the
+ * visible keys j of row i, with P_ij = exp(scale q_i . k_j - lse_i):
+ *   dP_ij = dout_i . v_j,  Delta_i = dout_i . o_i,  dS_ij = P_ij (dP_ij - Delta_i),
+ *   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,  dv_j = sum_i P_ij dout_i,
+ * dk and dv summed over the G = Hq / Hkv query heads that read a key/value head.
+ * P and dS enter the tensor-core products rounded to bf16; sums are fp32.
+ *
+ *  q, o, dout [B, Hq, N, d]  bf16 (device, read)
+ *  k, v       [B, Hkv, N, d] bf16 (device, read)
+ *  lse        [B, Hq, N]     fp32 (device, read): the lse attn_fwd returned
+ *  delta      [B, Hq, N]     fp32 (device): workspace, overwritten with Delta
+ *  dq         [B, Hq, N, d]  bf16 (device, written)
+ *  dk, dv     [B, Hkv, N, d] bf16 (device, written)
+ *  B*Hq <= 65535; N >= 1; d 64 or 128 (else ATTN_ERR_UNSUPPORTED); causal 0/1
+ *  (query i sees keys j <= i); scale finite and > 0. Outputs must not overlap
+ *  the inputs. Three launches on `stream`: Delta, then dk/dv (one block per
+ *  128-key tile and key/value head), then dq (one block per 128-row query tile
+ *  and query head).
+ */
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dout, float* delta, void* dq, void* dk, void* dv,
+                       int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                       attn_stream_t stream);
+
+/*
  * attn_fwd_f16, attn_decode_splitkv_f16, attn_combine_f16 — the same three calls
  * for IEEE fp16 inputs (the pages list FP16 beside BF16 among the supported
  * dtypes: "1-Flash-Attention.md", "使用注意事项"). Arguments, layouts, checks and

@@ -275,8 +275,6 @@ int oracle_decode_partials(int dtype, const void* q, const void* k, const void* 
     return 0;
 }
 
-// Logsumexp-weighted merge: M = max_s lse_s, w_s = exp(lse_s - M),
-// O = sum_s w_s O_s / sum_s w_s, LSE = M + ln sum_s w_s.
 // Gradients of the scalar sum(dO * O) with respect to Q, K and V, from the
 // definition (backward pass; the forward's LSE is recomputed, not taken from
 // the GPU): for the visible keys j of row i, with P the softmax of the row,
@@ -346,6 +344,8 @@ int oracle_widen(int dtype, const void* x, int64_t n, double* out) {
     return 0;
 }
 
+// Logsumexp-weighted merge: M = max_s lse_s, w_s = exp(lse_s - M),
+// O = sum_s w_s O_s / sum_s w_s, LSE = M + ln sum_s w_s.
 int oracle_combine(const double* o_part, const double* lse_part, int B, int Hq, int num_splits,
                    int d, double* o, double* lse) {
     if (B < 1 || Hq < 1 || num_splits < 1 || d < 1) return 1;

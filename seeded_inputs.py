@@ -41,6 +41,13 @@ def make_qkv(seed: int, B: int, Hq: int, Hkv: int, N: int, d: int, q_mult: float
     return q.contiguous(), k.contiguous(), v.contiguous()
 
 
+def make_dout(seed: int, B: int, Hq: int, N: int, d: int, dtype=torch.bfloat16):
+    """Output gradient for the backward pass: dO [B,Hq,N,d], N(0,1) rounded to
+    the input type, from its own generator (seed independent of q, k, v)."""
+    gen = torch.Generator().manual_seed(seed)
+    return _randn_bf16(gen, (B, Hq, N, d), dtype).contiguous()
+
+
 def make_decode(seed: int, B: int, Hq: int, Hkv: int, L: int, d: int, pin: bool = False, dtype=torch.bfloat16):
     """Single-query decode inputs: q [B,Hq,d], k/v [B,Hkv,L,d], CPU tensors (bf16, or fp16).
 

@@ -207,3 +207,24 @@ def test_decode_chunk_rule():
     assert decode_chunk(100, 64) == 128
     assert decode_chunk(1, 1) == 128
     assert decode_chunk(131072, 5) == 26240
+
+
+def _bwd(lib, q=16, k=32, v=48, o=64, lse=80, do=96, delta=112, dq=128, dk=144, dv=160, B=1, Hq=2, Hkv=1,
+         N=8, d=64, causal=0, scale=0.125):
+    P = ctypes.c_void_p
+    lib.attn_bwd.restype = ctypes.c_int
+    return lib.attn_bwd(P(q), P(k), P(v), P(o), P(lse), P(do), P(delta), P(dq), P(dk), P(dv), B, Hq, Hkv, N, d,
+                        causal, ctypes.c_float(scale), None)
+
+
+@pytest.mark.parametrize("kw", [dict(q=0), dict(k=0), dict(v=0), dict(o=0), dict(lse=0), dict(do=0),
+                                dict(delta=0), dict(dq=0), dict(dk=0), dict(dv=0), dict(dq=136), dict(lse=84),
+                                dict(B=0), dict(N=0), dict(Hq=3, Hkv=2), dict(causal=2), dict(scale=0.0),
+                                dict(scale=float("nan")), dict(B=2, Hq=40000, Hkv=40000)])
+def test_bwd_rejects_invalid(lib, kw):
+    assert _bwd(lib, **kw) == INVALID
+
+
+@pytest.mark.parametrize("d", [0, 32, 96, 256])
+def test_bwd_rejects_unsupported_head_dim(lib, d):
+    assert _bwd(lib, d=d) == UNSUPPORTED
