@@ -80,10 +80,15 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdParams p, long 
 // Shared skeleton of the two tile kernels. One block owns a fixed pair of
 // tiles (A_fix, B_fix: K and V for dK/dV; Q and dO for dQ) and streams pairs of
 // tiles (S_a, S_b: Q and dO; K and V) through two buffers. Per step:
-//   X = A_fix * S_a^T, Y = B_fix * S_b^T          (both M = 128, N = 128, K = D)
-//   element-wise: P from X and the row/column LSE, G = P o (Y - Delta) * scale
-//   acc1 += P * S_b, acc2 += G * S_a              (dK/dV: A from TMEM)
-// For dQ only acc2 (+= dS K) is kept.
+//   X = A_fix S_a^T, then Y = B_fix S_b^T          (M = 128, N = 128, K = D)
+//   element-wise, in two halves of 64 columns:
+//     P = exp2(X scale log2e - lse log2e)  (while Y is still being computed),
+//     G = P o (Y - Delta), both written back as bf16 over X and Y
+//   acc1 += P S_b, acc2 += G S_a                    (A from TMEM, B MN-major)
+// The accumulating MMAs of the first half run while the second half is being
+// computed. For dQ only acc2 (dS K) is kept. scale multiplies acc2 once, in
+// the epilogue. Steps whose tile holds no masked element (off the causal
+// diagonal, inside the sequence) skip the mask.
 // TMEM: X [0, 128), Y [128, 256), acc1 [256, 256 + D), acc2 [256 + D, 256 + 2D).
 template <int D, bool CAUSAL, bool DKDV>
 __global__ void __launch_bounds__(192, 1)
@@ -97,17 +102,19 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* sFA = smem;
     uint8_t* sFB = sFA + C::TILE_BYTES;
     uint8_t* sS = sFB + C::TILE_BYTES;  // [2 buffers][S_a, S_b]
-    float* sL = reinterpret_cast<float*>(sS + 4 * C::TILE_BYTES);  // [2 buffers][lse*log2e, delta][128]
+    // [2 buffers][-lse log2e, -Delta][128]: per streamed query row (dK/dV only)
+    float* sL = reinterpret_cast<float*>(sS + 4 * C::TILE_BYTES);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sL + 4 * BT);
     uint64_t* fix_full = bars;       // the fixed tiles loaded
     uint64_t* st_full = bars + 1;    // [2] streamed tiles of a buffer loaded
     uint64_t* st_empty = bars + 3;   // [2] streamed tiles of a buffer read by every MMA
-    uint64_t* xy_full = bars + 5;    // X and Y complete
-    uint64_t* pg_full = bars + 6;    // P and G written (4 warp arrivals)
-    uint64_t* l_ready = bars + 7;    // [2] lse/delta of a buffer staged (4 warp arrivals)
-    uint64_t* l_free = bars + 9;     // [2] lse/delta of a buffer read (4 warp arrivals)
-    uint64_t* fin = bars + 11;       // every MMA done
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12);
+    uint64_t* x_full = bars + 5;     // X complete
+    uint64_t* y_full = bars + 6;     // Y complete
+    uint64_t* pg_half = bars + 7;    // [2] P and G of a half written (4 warp arrivals)
+    uint64_t* l_ready = bars + 9;    // [2] lse/Delta of a buffer staged (4 warp arrivals)
+    uint64_t* l_free = bars + 11;    // [2] lse/Delta of a buffer read (4 warp arrivals)
+    uint64_t* fin = bars + 13;       // every MMA done
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -131,11 +138,12 @@ __global__ void __launch_bounds__(192, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&st_full[i], 2 * C::CHUNKS);
             mbar_init(&st_empty[i], 1);
+            mbar_init(&pg_half[i], 4);
             mbar_init(&l_ready[i], 4);
             mbar_init(&l_free[i], 4);
         }
-        mbar_init(xy_full, 1);
-        mbar_init(pg_full, 4);
+        mbar_init(x_full, 1);
+        mbar_init(y_full, 1);
         mbar_init(fin, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -206,29 +214,40 @@ __global__ void __launch_bounds__(192, 1)
                 ok = mbar_wait(&st_full[bu], (s >> 1) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                // X = A_fix S_a^T, Y = B_fix S_b^T (after the previous step's
-                // accumulating MMAs have read X and Y: issue order)
+                // X = A_fix S_a^T, then Y = B_fix S_b^T. Issued after the previous
+                // step's accumulating MMAs, which read P and G from these columns:
+                // the tensor pipe's issue order keeps them intact until read.
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
                     mma_ss(tX, make_sdesc_sw128(fa + koff, 16, 1024), make_sdesc_sw128(sa + koff, 16, 1024), idesc_xy,
                            kk > 0 ? 1u : 0u);
+                }
+                tc_commit(x_full);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
                     mma_ss(tY, make_sdesc_sw128(fb + koff, 16, 1024), make_sdesc_sw128(sb + koff, 16, 1024), idesc_xy,
                            kk > 0 ? 1u : 0u);
                 }
-                tc_commit(xy_full);
-                ok = mbar_wait_spin(pg_full, s & 1, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                // acc1 += P S_b (dK/dV only: dV += P^T dO), acc2 += G S_a (dK += dS^T Q,
-                // or dQ += dS K); A from TMEM (bf16 packed over X / Y), B MN-major
+                tc_commit(y_full);
+                // acc1 += P S_b (dV += P^T dO), acc2 += G S_a (dK += dS^T Q, or
+                // dQ += dS K), 64 streamed rows per half as each half lands
 #pragma unroll
-                for (int kk = 0; kk < BT / 16; ++kk) {
-                    const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                    if (DKDV)
-                        mma_ts(tA1, tX + kk * 8, make_sdesc_sw128(sb + kk * 16 * 128, BT * 128, 1024), idesc_acc, acc);
-                    mma_ts(tA2, tY + kk * 8, make_sdesc_sw128(sa + kk * 16 * 128, BT * 128, 1024), idesc_acc, acc);
+                for (int h = 0; h < 2; ++h) {
+                    ok = mbar_wait_spin(&pg_half[h], s & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = h * (BT / 32); kk < (h + 1) * (BT / 32); ++kk) {
+                        const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                        if (DKDV)
+                            mma_ts(tA1, tX + kk * 8, make_sdesc_sw128(sb + kk * 16 * 128, BT * 128, 1024), idesc_acc,
+                                   acc);
+                        mma_ts(tA2, tY + kk * 8, make_sdesc_sw128(sa + kk * 16 * 128, BT * 128, 1024), idesc_acc, acc);
+                    }
                 }
+                if (!ok) break;
                 tc_commit(&st_empty[bu]);
             }
             tc_commit(fin);
@@ -240,79 +259,125 @@ __global__ void __launch_bounds__(192, 1)
         const int row = warp * 32 + lane;  // TMEM lane: key (dK/dV) or query row (dQ)
         const uint32_t lb = tmem + (uint32_t(warp * 32) << 16);
         const uint32_t tX = lb, tY = lb + 128, tA1 = lb + 256, tA2 = lb + 256 + D;
-        const float c2 = p.scale_log2;
+        const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
         const float LOG2E = 1.4426950408889634f;
-        bool ok = nsteps > 0;
-        // this thread's own row: lse and delta (dQ: fixed query row)
-        float my_l2 = INFINITY, my_delta = 0.f;
-        if (!DKDV) {
-            const int qr = tile * BT + row;
-            if (qr < p.N) {
-                my_l2 = p.lse[static_cast<size_t>(b * p.Hq + hfix) * p.N + qr] * LOG2E;
-                my_delta = p.delta[static_cast<size_t>(b * p.Hq + hfix) * p.N + qr];
-            }
-        }
         const int fixed_pos = tile * BT + row;  // this thread's key (dK/dV) or query row (dQ)
-        for (int s = 0; ok && s < nsteps; ++s) {
-            const int bu = s & 1;
+        // dQ: this thread's own row's -lse log2e and -Delta (rows past the end: P = 0)
+        float nl2_row = -INFINITY, ndl_row = 0.f;
+        if (!DKDV && fixed_pos < p.N) {
+            const size_t r = static_cast<size_t>(b * p.Hq + hfix) * p.N + fixed_pos;
+            nl2_row = -p.lse[r] * LOG2E;
+            ndl_row = -p.delta[r];
+        }
+        // dK/dV: -lse log2e and -Delta of the streamed query rows, staged in
+        // shared memory one step ahead (each thread one row)
+        auto stage_load = [&](int s, float* nl2, float* ndl) {
             int plane, trow;
             step_src(s, &plane, &trow);
-            float* lsb = sL + bu * 2 * BT;  // per streamed query row: lse*log2e, then delta
-            if (DKDV) {
-                // stage the streamed query rows' lse and delta (column values)
-                if (s >= 2 && !__all_sync(0xffffffffu, mbar_wait(&l_free[bu], ((s >> 1) - 1) & 1, abort_flag))) {
-                    ok = false;
-                    break;
-                }
-                const int qr = trow + row;
-                lsb[row] = qr < p.N ? p.lse[static_cast<size_t>(plane) * p.N + qr] * LOG2E : INFINITY;
-                lsb[BT + row] = qr < p.N ? p.delta[static_cast<size_t>(plane) * p.N + qr] : 0.f;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&l_ready[bu]);
-                if (!__all_sync(0xffffffffu, mbar_wait(&l_ready[bu], (s >> 1) & 1, abort_flag))) {
-                    ok = false;
-                    break;
-                }
+            const int qr = trow + row;
+            const size_t r = static_cast<size_t>(plane) * p.N + qr;
+            *nl2 = qr < p.N ? -p.lse[r] * LOG2E : -INFINITY;
+            *ndl = qr < p.N ? -p.delta[r] : 0.f;
+        };
+        auto stage_store = [&](int s, float nl2, float ndl) {
+            float* lsb = sL + (s & 1) * 2 * BT;
+            lsb[row] = nl2;
+            lsb[BT + row] = ndl;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&l_ready[s & 1]);
+        };
+        bool ok = nsteps > 0;
+        float pre_nl2 = 0.f, pre_ndl = 0.f;
+        if (DKDV && ok) {
+            stage_load(0, &pre_nl2, &pre_ndl);
+            stage_store(0, pre_nl2, pre_ndl);
+        }
+        for (int s = 0; ok && s < nsteps; ++s) {
+            int plane, trow;
+            step_src(s, &plane, &trow);
+            if (DKDV && s + 1 < nsteps) stage_load(s + 1, &pre_nl2, &pre_ndl);
+            const float* lsb = sL + (s & 1) * 2 * BT;
+            if (DKDV && !__all_sync(0xffffffffu, mbar_wait(&l_ready[s & 1], (s >> 1) & 1, abort_flag))) {
+                ok = false;
+                break;
             }
-            if (!__all_sync(0xffffffffu, mbar_wait(xy_full, s & 1, abort_flag))) {
+            // visible columns of this thread's row: lo <= col < hi
+            // (dK/dV: query = trow + col >= key; dQ: key = trow + col <= query)
+            const int hi = DKDV ? p.N - trow : (CAUSAL ? min(p.N, fixed_pos + 1) : p.N) - trow;
+            const int lo = (DKDV && CAUSAL) ? fixed_pos - trow : 0;
+            const bool need_mask = trow + BT > p.N || (CAUSAL && trow == tile * BT);
+            if (!__all_sync(0xffffffffu, mbar_wait(x_full, s & 1, abort_flag))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                uint32_t xs[64], ys[64];
-                tmem_ld64(tX + h * 64, xs);
-                tmem_ld64(tY + h * 64, ys);
-                uint32_t pk[32], gk[32];
+                // P of 64 columns from X
+                float pf[64];
+                {
+                    uint32_t xs[64];
+                    tmem_ld64(tX + h * 64, xs);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    float pv[2], gv[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int col = h * 64 + 2 * i + e;  // streamed row (dK/dV) or key (dQ) in the tile
-                        const int other = trow + col;
-                        const float l2 = DKDV ? lsb[col] : my_l2;
-                        const float dl = DKDV ? lsb[BT + col] : my_delta;
-                        // visible: query row >= key (causal), and both inside the sequence
-                        const int qpos = DKDV ? other : fixed_pos, kpos = DKDV ? fixed_pos : other;
-                        const bool vis = other < p.N && (!CAUSAL || qpos >= kpos);
-                        const float pr = vis ? ex2_approx(__uint_as_float(xs[2 * i + e]) * c2 - l2) : 0.f;
-                        pv[e] = pr;
-                        gv[e] = pr * (__uint_as_float(ys[2 * i + e]) - dl) * p.scale;
+                    for (int i = 0; i < 32; ++i) {
+                        const int col = h * 64 + 2 * i;
+                        const float2 nl2 =
+                            DKDV ? *reinterpret_cast<const float2*>(lsb + col) : make_float2(nl2_row, nl2_row);
+                        const float2 a =
+                            ffma2(make_float2(__uint_as_float(xs[2 * i]), __uint_as_float(xs[2 * i + 1])), c2, nl2);
+                        pf[2 * i] = ex2_approx(a.x);
+                        pf[2 * i + 1] = ex2_approx(a.y);
                     }
-                    pk[i] = pack_bf16x2(pv[0], pv[1]);
-                    gk[i] = pack_bf16x2(gv[0], gv[1]);
                 }
-                if (DKDV) tmem_st32(tX + h * 32, pk);
-                tmem_st32(tY + h * 32, gk);
+                if (need_mask) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        const int col = h * 64 + i;
+                        if (col < lo || col >= hi) pf[i] = 0.f;
+                    }
+                }
+                if (h == 0 && !__all_sync(0xffffffffu, mbar_wait(y_full, s & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                // G = P (Y - Delta), 32 columns at a time
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    uint32_t ys[32], pk[16], gk[16];
+                    tmem_ld32(tY + h * 64 + q * 32, ys);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int j = q * 32 + 2 * i;  // column inside the half
+                        const float2 ndl = DKDV ? *reinterpret_cast<const float2*>(lsb + BT + h * 64 + j)
+                                                : make_float2(ndl_row, ndl_row);
+                        const float2 t =
+                            fadd2(make_float2(__uint_as_float(ys[2 * i]), __uint_as_float(ys[2 * i + 1])), ndl);
+                        const float2 g = fmul2(make_float2(pf[j], pf[j + 1]), t);
+                        pk[i] = pack_bf16x2(pf[j], pf[j + 1]);
+                        gk[i] = pack_bf16x2(g.x, g.y);
+                    }
+                    if (DKDV) tmem_st16(tX + h * 32 + q * 16, pk);
+                    tmem_st16(tY + h * 32 + q * 16, gk);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&pg_half[h]);
             }
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if (DKDV) mbar_arrive(&l_free[bu]);
-                mbar_arrive(pg_full);
+            if (!ok) break;
+            if (DKDV) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&l_free[s & 1]);
+                if (s + 1 < nsteps) {
+                    // buffer (s + 1) & 1 was last read in step s - 1
+                    if (s >= 1 &&
+                        !__all_sync(0xffffffffu, mbar_wait(&l_free[(s + 1) & 1], ((s - 1) >> 1) & 1, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    stage_store(s + 1, pre_nl2, pre_ndl);
+                }
             }
         }
         // epilogue: the accumulators (dV, dK; or dQ) to bf16 rows of the output
@@ -326,6 +391,7 @@ __global__ void __launch_bounds__(192, 1)
             for (int which = 0; which < (DKDV ? 2 : 1); ++which) {
                 __nv_bfloat16* dst = (DKDV ? (which == 0 ? p.dv : p.dk) : p.dq) + out_row * D;
                 const uint32_t src = DKDV ? (which == 0 ? tA1 : tA2) : tA2;
+                const float f = (DKDV && which == 0) ? 1.f : p.scale;  // dK, dQ carry the scale
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t r3[32];
@@ -334,10 +400,10 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                         for (int i = 0; i < 32; i += 8)
                             *reinterpret_cast<uint4*>(dst + c * 32 + i) = make_uint4(
-                                pack_bf16x2(__uint_as_float(r3[i]), __uint_as_float(r3[i + 1])),
-                                pack_bf16x2(__uint_as_float(r3[i + 2]), __uint_as_float(r3[i + 3])),
-                                pack_bf16x2(__uint_as_float(r3[i + 4]), __uint_as_float(r3[i + 5])),
-                                pack_bf16x2(__uint_as_float(r3[i + 6]), __uint_as_float(r3[i + 7])));
+                                pack_bf16x2(__uint_as_float(r3[i]) * f, __uint_as_float(r3[i + 1]) * f),
+                                pack_bf16x2(__uint_as_float(r3[i + 2]) * f, __uint_as_float(r3[i + 3]) * f),
+                                pack_bf16x2(__uint_as_float(r3[i + 4]) * f, __uint_as_float(r3[i + 5]) * f),
+                                pack_bf16x2(__uint_as_float(r3[i + 6]) * f, __uint_as_float(r3[i + 7]) * f));
                     }
                 }
             }
