@@ -48,6 +48,12 @@ def _bind(lib):
     lib.oracle_widen.restype = I
     lib.oracle_attention_backward.argtypes = [I, P, P, P, P, I, I, I, I, I, I, D, P, P, P, I]
     lib.oracle_attention_backward.restype = I
+    lib.oracle_quant_fp8.argtypes = [I, P, I, I, I, I, P, P]
+    lib.oracle_quant_fp8.restype = I
+    lib.oracle_e4m3_decode.argtypes = [P, L, P]
+    lib.oracle_e4m3_decode.restype = I
+    lib.oracle_e4m3_encode.argtypes = [P, L, P]
+    lib.oracle_e4m3_encode.restype = I
     return lib
 
 
@@ -183,3 +189,45 @@ def attention_backward(q, k, v, dout, causal: bool, scale: float, nthreads: int 
                                            int(causal), float(scale), _ptr(dq), _ptr(dk), _ptr(dv), nthreads)
     _check(rc, "attention_backward")
     return dq, dk, dv
+
+
+def e4m3_encode(x, plant: int = 0):
+    """E4M3 codes (uint8) of a float32 tensor: nearest value, ties to even,
+    saturated at +-448."""
+    x = x.to(torch.float32).contiguous()
+    out = torch.empty(x.shape, dtype=torch.uint8)
+    _check(_load(plant).oracle_e4m3_encode(_ptr(x), x.numel(), _ptr(out)), "e4m3_encode")
+    return out
+
+
+def e4m3_decode(codes):
+    """Values (float64) of E4M3 codes."""
+    codes = codes.contiguous()
+    assert codes.dtype == torch.uint8
+    out = torch.empty(codes.shape, dtype=torch.float64)
+    _check(_load().oracle_e4m3_decode(_ptr(codes), codes.numel(), _ptr(out)), "e4m3_decode")
+    return out
+
+
+def quant_fp8(x, per_plane: bool = False, plant: int = 0):
+    """Block quantisation of x [..., N, d] (bf16, f32 or f16) to E4M3: returns
+    (codes uint8 of x's shape, scales fp32 [..., ceil(N / 128)]), one scale per
+    128-row block (per_plane: one per [N, d] plane, repeated per block)."""
+    x = x.contiguous()
+    *lead, N, d = x.shape
+    planes = 1
+    for n in lead:
+        planes *= n
+    nblk = (N + 127) // 128
+    codes = torch.empty(x.shape, dtype=torch.uint8)
+    scales = torch.empty(*lead, nblk, dtype=torch.float32)
+    _check(_load(plant).oracle_quant_fp8(_DT[x.dtype], _ptr(x), planes, N, d, int(per_plane), _ptr(codes),
+                                         _ptr(scales)), "quant_fp8")
+    return codes, scales
+
+
+def dequant_fp8(codes, scales):
+    """float64 values codes stand for: e4m3 value x the scale of the row's block."""
+    N = codes.shape[-2]
+    rep = scales.to(torch.float64).repeat_interleave(128, dim=-1)[..., :N]
+    return e4m3_decode(codes) * rep.unsqueeze(-1)

@@ -25,6 +25,9 @@
 //                                   the direct definition
 //  oracle_decode_partials           per-split partial (O_s, lse_s)
 //  oracle_combine                   logsumexp-weighted merge of partials
+//  oracle_attention_backward        dQ, dK, dV from the definition
+//  oracle_quant_fp8                 block quantisation to FP8 (E4M3) codes
+//  oracle_e4m3_decode               FP8 (E4M3) code -> value
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -73,6 +76,52 @@ inline double load_elem(int dtype, const void* base, int64_t idx) {
             return f;
         }
     }
+}
+
+// FP8 E4M3 (the "fn" variant: 1 sign bit, 4 exponent bits with bias 7, 3
+// fraction bits, no infinities, S.1111.111 is NaN, largest finite 448), from
+// the format's definition: exponent field 0 holds zero and the subnormals
+// (fraction * 2^-9); otherwise (1 + fraction / 8) * 2^(e - 7).
+inline double e4m3_value(uint8_t c) {
+    const int sign = c >> 7, e = (c >> 3) & 15, f = c & 7;
+    double mag;
+    if (e == 15 && f == 7)
+        mag = std::numeric_limits<double>::quiet_NaN();
+    else if (e == 0)
+        mag = std::ldexp(static_cast<double>(f), -9);
+    else
+        mag = std::ldexp(1.0 + f / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+// Nearest E4M3 value to a finite float, ties to the even code, magnitudes past
+// 448 saturated to 448. The step between neighbours is 2^(E-3) in the binade
+// [2^E, 2^(E+1)) for E >= -6, and 2^-9 below 2^-6 (the subnormals); dividing by
+// the step is exact, so one rounding to an integer count of steps decides it.
+inline uint8_t e4m3_code(float x) {
+    const uint8_t sign = std::signbit(x) ? 0x80 : 0x00;
+    const double a = std::fabs(static_cast<double>(x));
+    if (a >= 448.0) return sign | 0x7E;  // saturate (448 = 1.75 * 2^8)
+    int E = a > 0.0 ? std::ilogb(a) : -7;
+    if (E < -6) E = -6;
+    const double step = std::ldexp(1.0, E - 3);
+    double n = a / step;
+    double r = std::floor(n);
+    const double frac = n - r;
+    if (kPlant == 10) {
+        // 10: rounds toward zero
+    } else if (frac > 0.5 || (frac == 0.5 && std::fmod(r, 2.0) != 0.0)) {
+        r += 1.0;
+    }
+    // r steps of 2^(E-3): r in [8, 16] for a normal binade (16 carries into
+    // the next binade), r in [0, 8] for the subnormal range
+    const double v = r * step;
+    if (v == 0.0) return sign;
+    if (v >= 448.0) return sign | 0x7E;
+    int Ev = std::ilogb(v);
+    if (Ev < -6) return sign | static_cast<uint8_t>(r);  // subnormal: fraction = r
+    const int frac_bits = static_cast<int>(std::ldexp(v, -Ev) * 8.0) - 8;
+    return sign | static_cast<uint8_t>(((Ev + 7) << 3) | frac_bits);
 }
 
 struct Problem {
@@ -365,6 +414,61 @@ int oracle_combine(const double* o_part, const double* lse_part, int B, int Hq, 
         for (int t = 0; t < d; ++t) o[bh * d + t] /= wsum;
         lse[bh] = M + std::log(wsum);
     }
+    return 0;
+}
+
+// FP8 block quantisation (FlashAttention-3 page: FP8 through block
+// quantisation). Reading taken where the page gives no detail: one fp32 scale
+// per block of 128 consecutive rows of a (batch, head) plane, or one per plane
+// when per_plane != 0; s = amax / 448 (amax = largest |x| in the block, s = 1
+// for an all-zero block), computed in fp32, and code = E4M3(x / s) with the
+// division in fp32, ties to even. The value a code stands for is
+// e4m3_value(code) * s.
+//   x      [planes, N, d] in dtype (bf16, f32 or f16)
+//   codes  [planes, N, d] uint8 (written)
+//   scales [planes, ceil(N / 128)] fp32 (written)
+int oracle_quant_fp8(int dtype, const void* x, int planes, int N, int d, int per_plane, uint8_t* codes,
+                     float* scales) {
+    if (x == nullptr || codes == nullptr || scales == nullptr || planes < 1 || N < 1 || d < 1 ||
+        dtype < IN_BF16 || dtype > IN_F16)
+        return 1;
+    const int nblk = (N + 127) / 128;
+    std::vector<float> amax(nblk);
+    for (int64_t pl = 0; pl < planes; ++pl) {
+        for (int bk = 0; bk < nblk; ++bk) {
+            float m = 0.f;
+            for (int64_t n = bk * 128; n < std::min<int64_t>(N, (bk + 1) * 128); ++n)
+                for (int t = 0; t < d; ++t)
+                    m = std::max(m, static_cast<float>(std::fabs(load_elem(dtype, x, (pl * N + n) * d + t))));
+            amax[bk] = m;
+        }
+        float plane_max = 0.f;
+        for (float m : amax) plane_max = std::max(plane_max, m);
+        for (int bk = 0; bk < nblk; ++bk) {
+            const float m = per_plane ? plane_max : amax[bk];
+            const float sc = m > 0.f ? m / 448.0f : 1.0f;
+            scales[pl * nblk + bk] = sc;
+            for (int64_t n = bk * 128; n < std::min<int64_t>(N, (bk + 1) * 128); ++n)
+                for (int t = 0; t < d; ++t) {
+                    const int64_t i = (pl * N + n) * d + t;
+                    codes[i] = e4m3_code(static_cast<float>(load_elem(dtype, x, i)) / sc);
+                }
+        }
+    }
+    return 0;
+}
+
+// Values of n E4M3 codes.
+int oracle_e4m3_decode(const uint8_t* codes, int64_t n, double* out) {
+    if (codes == nullptr || out == nullptr || n < 0) return 1;
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_value(codes[i]);
+    return 0;
+}
+
+// E4M3 codes of n floats (exposes the rounding to the pin tests).
+int oracle_e4m3_encode(const float* x, int64_t n, uint8_t* out) {
+    if (x == nullptr || out == nullptr || n < 0) return 1;
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_code(x[i]);
     return 0;
 }
 

@@ -10,7 +10,8 @@ recurrence of the "递归计算softmax" section of "1-Flash-Attention.md").
 The mutation test at the bottom builds oracle variants with one planted
 mistake each (a dropped scale, a wrong GQA grouping, a causal off-by-one, a
 log2 LSE, a missing rescale, a plain-average merge, a transposed K, a dropped
-key, unnormalised partials) and checks that at least one pin fails on each.
+key, unnormalised partials, E4M3 rounding toward zero) and checks that at
+least one pin fails on each.
 """
 import math
 
@@ -243,10 +244,60 @@ def pin_row_sampling(plant=0):
     assert torch.equal(orr, o.reshape(-1, 4)[rows]) and torch.equal(lr, lse.reshape(-1)[rows])
 
 
+def pin_e4m3_codec_matches_torch(plant=0):
+    """E4M3 values of all 256 codes, and the nearest-even rounding of floats
+    (random values across the range, and every exact midpoint between two
+    neighbouring values), against torch's float8_e4m3fn conversion."""
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64)
+    mine = oracle.e4m3_decode(codes)
+    nan = torch.isnan(ref)
+    assert torch.isnan(mine[nan]).all() and torch.equal(mine[~nan], ref[~nan])
+    g = torch.Generator().manual_seed(60)
+    x = torch.cat([torch.randn(20000, generator=g) * 60, torch.randn(20000, generator=g) * 0.02,
+                   (torch.rand(20000, generator=g) * 2 - 1) * 448]).clamp(-448, 448)
+    pos = torch.unique(ref[~nan].abs()).sort().values
+    mid = ((pos[1:] + pos[:-1]) / 2).to(torch.float32)
+    x = torch.cat([x, mid, -mid])
+    assert torch.equal(oracle.e4m3_encode(x, plant=plant), x.to(torch.float8_e4m3fn).view(torch.uint8))
+    # saturation past the largest finite value
+    big = torch.tensor([448.0, 470.0, 1e6, -1e6])
+    assert oracle.e4m3_decode(oracle.e4m3_encode(big, plant=plant)).tolist() == [448.0, 448.0, 448.0, -448.0]
+
+
+def pin_quant_fp8_blocks(plant=0):
+    """Block quantisation: scale = amax / 448 in fp32 per 128-row block (or per
+    plane), codes = torch's E4M3 rounding of x / scale in fp32; the largest
+    element of a block lands on +-448 exactly; an all-zero block has scale 1."""
+    g = torch.Generator().manual_seed(61)
+    x = (torch.randn(2, 3, 300, 64, generator=g) * torch.tensor([0.01, 1.0, 30.0]).view(1, 3, 1, 1)).to(torch.bfloat16)
+    x[1, 2, 128:256] = 0
+    for per_plane in (False, True):
+        codes, scales = oracle.quant_fp8(x, per_plane=per_plane, plant=plant)
+        xf = x.float()
+        blocks = [xf[..., i:i + 128, :].abs().amax(dim=(-1, -2)) for i in range(0, 300, 128)]
+        amax = torch.stack(blocks, dim=-1)
+        if per_plane:
+            amax = amax.amax(dim=-1, keepdim=True).expand_as(amax)
+        want = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+        assert torch.equal(scales, want)
+        rep = scales.repeat_interleave(128, dim=-1)[..., :300].unsqueeze(-1)
+        assert torch.equal(codes, (xf / rep).to(torch.float8_e4m3fn).view(torch.uint8))
+        deq = oracle.dequant_fp8(codes, scales)
+        if not per_plane:
+            top = deq.abs().amax(dim=-1)
+            for i, s0 in enumerate(range(0, 300, 128)):
+                blk = top[..., s0:s0 + 128].amax(dim=-1)
+                nz = amax[..., i] > 0
+                assert torch.equal(blk[nz], (448.0 * scales[..., i].double())[nz])
+    assert torch.equal(oracle.quant_fp8(x)[1][1, 2, 1], torch.tensor(1.0))
+
+
 PINS = [pin_probs_are_distributions, pin_constant_v, pin_causal_first_row, pin_single_key,
         pin_two_keys_closed_form, pin_identical_keys, pin_library_sdpa, pin_brute_force_tiny,
         pin_blockwise_equals_direct, pin_invariants, pin_decode_and_combine,
-        pin_bf16_inputs_widen_exactly, pin_fp16_inputs_widen_exactly, pin_row_sampling]
+        pin_bf16_inputs_widen_exactly, pin_fp16_inputs_widen_exactly, pin_row_sampling,
+        pin_e4m3_codec_matches_torch, pin_quant_fp8_blocks]
 
 
 def test_backward_matches_autograd():
@@ -294,7 +345,7 @@ def test_pin(pin):
 
 PLANTS = {1: "scale dropped", 2: "GQA head h % Hkv", 3: "causal off by one", 4: "LSE in log2",
           5: "recurrence without rescale", 6: "merge by plain average", 7: "K read transposed",
-          8: "one key dropped", 9: "partials not normalised"}
+          8: "one key dropped", 9: "partials not normalised", 10: "E4M3 rounding toward zero"}
 
 
 @pytest.mark.parametrize("plant", sorted(PLANTS), ids=[PLANTS[p] for p in sorted(PLANTS)])
