@@ -58,6 +58,10 @@ def _load():
     lib.attn_merge.restype = I
     lib.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.attn_bwd.restype = I
+    lib.attn_quant_fp8.argtypes = [P, P, P, I, I, I, I, I, P]
+    lib.attn_quant_fp8.restype = I
+    lib.attn_fwd_fp8.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.attn_fwd_fp8.restype = I
     return lib
 
 
@@ -148,6 +152,44 @@ def attn_bwd(q, k, v, o, lse, dout, delta, dq, dk, dv, causal: bool, scale: floa
     _check(_lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(delta), _ptr(dq),
                          _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream)),
            "attn_bwd")
+
+
+def attn_quant_fp8(x, codes, scales, per_plane: bool = False, transpose: bool = False, stream=None):
+    """E4M3 block quantisation of x [..., N, d] bf16: codes uint8 [..., N, d]
+    (transpose: [..., d, Np], Np = 128 * ceil(N / 128)), scales fp32
+    [..., ceil(N / 128)]."""
+    _need(x, torch.bfloat16, "x")
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.float32, "scales")
+    *lead, N, d = x.shape
+    planes = 1
+    for n in lead:
+        planes *= n
+    nblk = -(-N // 128)
+    want = (*lead, d, nblk * 128) if transpose else tuple(x.shape)
+    if tuple(codes.shape) != want or tuple(scales.shape) != (*lead, nblk):
+        raise ValueError("attn_quant_fp8: inconsistent shapes")
+    _check(_lib.attn_quant_fp8(_ptr(x), _ptr(codes), _ptr(scales), planes, N, d, int(bool(per_plane)),
+                               int(bool(transpose)), _stream(stream)), "attn_quant_fp8")
+
+
+def attn_fwd_fp8(q8, k8, vt8, sq, sk, sv, o, lse, causal: bool, scale: float, stream=None):
+    """q8 [B,Hq,N,128], k8 [B,Hkv,N,128], vt8 [B,Hkv,128,Np] E4M3 codes (uint8) with
+    their scales; o [B,Hq,N,128] bf16, lse [B,Hq,N] fp32."""
+    for t, n in ((q8, "q8"), (k8, "k8"), (vt8, "vt8")):
+        _need(t, torch.uint8, n)
+    for t, n in ((sq, "sq"), (sk, "sk"), (sv, "sv"), (lse, "lse")):
+        _need(t, torch.float32, n)
+    _need(o, torch.bfloat16, "o")
+    B, Hq, N, d = q8.shape
+    Hkv = k8.shape[1]
+    nblk = -(-N // 128)
+    if (k8.shape != (B, Hkv, N, d) or vt8.shape != (B, Hkv, d, nblk * 128) or sq.shape != (B, Hq, nblk)
+            or sk.shape != (B, Hkv, nblk) or sv.shape != (B, Hkv, nblk) or o.shape != q8.shape
+            or lse.shape != (B, Hq, N)):
+        raise ValueError("attn_fwd_fp8: inconsistent shapes")
+    _check(_lib.attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(vt8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o), _ptr(lse),
+                             B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream)), "attn_fwd_fp8")
 
 
 def _dec(fn, name, dt, q, k, v, o_part, lse_part, num_splits, scale, stream):
@@ -258,6 +300,31 @@ def attention_backward(q, k, v, o, lse, dout, causal: bool = False, scale: float
     delta = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)
     attn_bwd(q, k, v, o, lse, dout, delta, dq, dk, dv, causal, scale, stream)
     return dq, dk, dv
+
+
+def quantize_fp8(x, per_plane: bool = False, transpose: bool = False, stream=None):
+    """Allocates and fills (codes, scales) for attn_quant_fp8."""
+    *lead, N, d = x.shape
+    nblk = -(-N // 128)
+    shape = (*lead, d, nblk * 128) if transpose else tuple(x.shape)
+    codes = torch.empty(shape, device=x.device, dtype=torch.uint8)
+    scales = torch.empty(*lead, nblk, device=x.device, dtype=torch.float32)
+    attn_quant_fp8(x, codes, scales, per_plane, transpose, stream)
+    return codes, scales
+
+
+def attention_fp8(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
+    """FP8 forward from bf16 q, k, v: quantises Q and K per 128-row block and V
+    per plane (transposed), then runs attn_fwd_fp8. Returns (o bf16, lse fp32)."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    q8, sq = quantize_fp8(q, stream=stream)
+    k8, sk = quantize_fp8(k, stream=stream)
+    vt8, sv = quantize_fp8(v, per_plane=True, transpose=True, stream=stream)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)
+    attn_fwd_fp8(q8, k8, vt8, sq, sk, sv, o, lse, causal, scale, stream)
+    return o, lse
 
 
 def decode(q, k, v, scale: float | None = None, num_splits: int | None = None, stream=None):

@@ -16,6 +16,7 @@
 #include "../../include/attn.h"
 #include "attn_fwd_sm100.cuh"
 #include "bwd_sm100.cuh"
+#include "fp8_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "merge_sm100.cuh"
 
@@ -55,6 +56,20 @@ bool make_map(CUtensorMap* map, const void* base, int D, int rows, int planes, i
     const cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, tma_type<E>(), 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// uint8 (E4M3 codes) tensor viewed as [planes, rows, inner] bytes with a
+// {128, 128, 1} box and 128-byte swizzle; rows past `rows` read as zero.
+bool make_map_u8(CUtensorMap* map, const void* base, int inner, int rows, int planes) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {cuuint64_t(inner), cuuint64_t(rows), cuuint64_t(planes)};
+    const cuuint64_t strides[2] = {cuuint64_t(inner), cuuint64_t(inner) * cuuint64_t(rows)};
+    const cuuint32_t box[3] = {128, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -302,6 +317,63 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d == 128) return causal ? launch_bwd<128, true>(tq, tk, tv, tdo, p, st) : launch_bwd<128, false>(tq, tk, tv, tdo, p, st);
     return causal ? launch_bwd<64, true>(tq, tk, tv, tdo, p, st) : launch_bwd<64, false>(tq, tk, tv, tdo, p, st);
+}
+
+attn_status_t attn_quant_fp8(const void* x, void* codes, float* scales, int planes, int N, int d, int per_plane,
+                             int transpose, attn_stream_t stream) {
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return ATTN_ERR_INVALID_ARG;
+    if (planes < 1 || N < 1 || (per_plane != 0 && per_plane != 1) || (transpose != 0 && transpose != 1))
+        return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    const int nblk = (N + 127) / 128;
+    if (planes > 65535) return ATTN_ERR_INVALID_ARG;
+    QuantParams p;
+    p.x = static_cast<const __nv_bfloat16*>(x);
+    p.codes = static_cast<uint8_t*>(codes);
+    p.scales = scales;
+    p.planes = planes; p.N = N; p.nblk = nblk; p.Np = nblk * 128; p.per_plane = per_plane;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid(nblk, planes);
+    if (d == 128) {
+        fp8_amax_kernel<128><<<grid, 256, 0, st>>>(p);
+        if (transpose) fp8_quant_kernel<128, true><<<grid, 256, 0, st>>>(p);
+        else fp8_quant_kernel<128, false><<<grid, 256, 0, st>>>(p);
+    } else {
+        fp8_amax_kernel<64><<<grid, 256, 0, st>>>(p);
+        if (transpose) fp8_quant_kernel<64, true><<<grid, 256, 0, st>>>(p);
+        else fp8_quant_kernel<64, false><<<grid, 256, 0, st>>>(p);
+    }
+    fp8_scales_kernel<<<(planes + 255) / 256, 256, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* sq, const float* sk,
+                           const float* sv, void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal,
+                           float scale, attn_stream_t stream) {
+    const void* ptrs[] = {q8, k8, vt8, sq, sk, sv, o, lse};
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || (causal != 0 && causal != 1) || !scale_ok(scale))
+        return ATTN_ERR_INVALID_ARG;
+    if (d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (static_cast<long long>(B) * Hq > 65535LL) return ATTN_ERR_INVALID_ARG;
+    const int nblk = (N + 127) / 128;
+    CUtensorMap tq, tk, tv;
+    if (!make_map_u8(&tq, q8, 128, N, B * Hq) || !make_map_u8(&tk, k8, 128, N, B * Hkv) ||
+        !make_map_u8(&tv, vt8, nblk * 128, 128, B * Hkv))
+        return ATTN_ERR_CUDA;
+    Fp8Params p;
+    p.sq = sq; p.sk = sk; p.sv = sv;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.nblk = nblk;
+    p.scale_log2 = scale * kLog2e;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    auto kern = causal ? attn_fwd_fp8_kernel<true> : attn_fwd_fp8_kernel<false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Fp8Cfg::SMEM_BYTES) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    kern<<<dim3(nblk, B * Hq), Fp8Cfg::NUM_THREADS, Fp8Cfg::SMEM_BYTES, st>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 int attn_decode_default_splits(int B, int Hq, int Hkv, int L) {

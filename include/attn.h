@@ -171,6 +171,42 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
                        attn_stream_t stream);
 
 /*
+ * attn_quant_fp8, attn_fwd_fp8 — the forward pass on FP8 (E4M3) inputs.
+ * FlashAttention-3 page: FP8 computation with block quantisation (incoherent
+ * processing, its other ingredient, is not provided). Reading of "block
+ * quantisation": one fp32 scale per block of 128 consecutive rows of a
+ * (batch, head) plane — or one per plane — s = amax / 448 with amax the
+ * largest |x| of the block (s = 1 for an all-zero block), code = E4M3(x / s),
+ * round to nearest even, IEEE fp32 division; the code stands for
+ * E4M3(code) * s.
+ *
+ * attn_quant_fp8 quantises x [planes, N, d] bf16 (device, read):
+ *  codes   transpose == 0: [planes, N, d] uint8; transpose == 1: [planes, d, Np]
+ *          uint8 with Np = 128 * ceil(N / 128), codes of keys >= N zero
+ *  scales  [planes, ceil(N / 128)] fp32 (written); with per_plane != 0 every
+ *          block of a plane gets the plane's scale
+ *  d 64 or 128 (else ATTN_ERR_UNSUPPORTED); planes <= 65535. Three launches.
+ *
+ * attn_fwd_fp8 computes O and LSE (as attn_fwd) from quantised inputs:
+ *  q8  [B, Hq, N, 128]  codes from attn_quant_fp8(q, ..., per_plane 0, transpose 0)
+ *  k8  [B, Hkv, N, 128] codes from attn_quant_fp8(k, ..., per_plane 0, transpose 0)
+ *  vt8 [B, Hkv, 128, Np] codes from attn_quant_fp8(v, ..., per_plane 1, transpose 1)
+ *  sq, sk, sv           the matching scales
+ *  o   [B, Hq, N, 128] bf16, lse [B, Hq, N] fp32 (written)
+ * S = Q8 K8^T runs on the tensor cores in E4M3 with fp32 accumulation and the
+ * block scales applied to the fp32 scores; P is rounded to E4M3 for the P V
+ * product (kept at most 2^8 by rescaling O whenever a row's maximum grows by
+ * more than 8 in log2 units); l sums the fp32 P. d must be 128 (else
+ * ATTN_ERR_UNSUPPORTED); B*Hq <= 65535; other checks as attn_fwd.
+ */
+attn_status_t attn_quant_fp8(const void* x, void* codes, float* scales, int planes, int N, int d,
+                             int per_plane, int transpose, attn_stream_t stream);
+attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* sq,
+                           const float* sk, const float* sv, void* o, float* lse,
+                           int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                           attn_stream_t stream);
+
+/*
  * attn_fwd_f16, attn_decode_splitkv_f16, attn_combine_f16 — the same three calls
  * for IEEE fp16 inputs (the pages list FP16 beside BF16 among the supported
  * dtypes: "1-Flash-Attention.md", "使用注意事项"). Arguments, layouts, checks and

@@ -228,3 +228,39 @@ def test_bwd_rejects_invalid(lib, kw):
 @pytest.mark.parametrize("d", [0, 32, 96, 256])
 def test_bwd_rejects_unsupported_head_dim(lib, d):
     assert _bwd(lib, d=d) == UNSUPPORTED
+
+
+def _quant8(lib, x=16, c=32, s=48, planes=2, N=100, d=128, per_plane=0, transpose=0):
+    P = ctypes.c_void_p
+    lib.attn_quant_fp8.restype = ctypes.c_int
+    return lib.attn_quant_fp8(P(x), P(c), P(s), planes, N, d, per_plane, transpose, None)
+
+
+def _fwd8(lib, q=16, k=32, v=48, sq=64, sk=80, sv=96, o=112, lse=128, B=1, Hq=2, Hkv=1, N=8, d=128, causal=0,
+          scale=0.125):
+    P = ctypes.c_void_p
+    lib.attn_fwd_fp8.restype = ctypes.c_int
+    return lib.attn_fwd_fp8(P(q), P(k), P(v), P(sq), P(sk), P(sv), P(o), P(lse), B, Hq, Hkv, N, d, causal,
+                            ctypes.c_float(scale), None)
+
+
+@pytest.mark.parametrize("kw", [dict(x=0), dict(c=0), dict(s=0), dict(c=40), dict(planes=0), dict(N=0),
+                                dict(per_plane=2), dict(transpose=-1), dict(planes=70000)])
+def test_quant_fp8_rejects_invalid(lib, kw):
+    assert _quant8(lib, **kw) == INVALID
+
+
+@pytest.mark.parametrize("d", [0, 32, 96, 256])
+def test_quant_fp8_rejects_unsupported_head_dim(lib, d):
+    assert _quant8(lib, d=d) == UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw", [dict(q=0), dict(v=0), dict(sv=0), dict(o=0), dict(lse=8), dict(N=0),
+                                dict(Hq=3, Hkv=2), dict(causal=2), dict(scale=0.0), dict(B=2, Hq=40000, Hkv=40000)])
+def test_fwd_fp8_rejects_invalid(lib, kw):
+    assert _fwd8(lib, **kw) == INVALID
+
+
+@pytest.mark.parametrize("d", [64, 96, 256])
+def test_fwd_fp8_rejects_unsupported_head_dim(lib, d):
+    assert _fwd8(lib, d=d) == UNSUPPORTED
