@@ -1,4 +1,5 @@
-"""Exact attention on B200 (sm_100a): prefill forward, split-KV decode, combine.
+"""Exact attention on B200 (sm_100a): prefill forward, split-KV decode, combine,
+ring attention, backward pass, FP8 forward.
 
 Thin Python binding over the C ABI of ``_lib/libattn_b200.so`` (declared in
 ``include/attn.h``). The binding only marshals arguments: every step of the

@@ -11,6 +11,9 @@
  * page, the split-K combine step). Ring attention (context parallelism) shards a
  * long sequence across devices and merges each device's per-shard results the
  * same way (attn_fwd_f32, attn_merge; FlashAttention-3 page, RingAttention).
+ * The backward pass (attn_bwd) recomputes P from the saved log-sum-exp; the
+ * FP8 forward (attn_quant_fp8, attn_fwd_fp8) runs on block-quantised E4M3
+ * inputs (FlashAttention-3 page).
  *
  * Conventions shared by every call:
  *  - All tensors are dense, contiguous, row-major device buffers owned by the
