@@ -175,6 +175,42 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # ----------------------------------------------------------------- our arm --
 
+def measure_extra_paths(eab, q, k, v, o, lse, p, flush, stream, iters=10, warm=3):
+    """The backward pass and the FP8 forward on the prefill workload (causal),
+    each timed alone with CUDA events after the timed step (L2 flushed before
+    every launch); median of `iters` launches."""
+    def timed(fn):
+        for _ in range(warm):
+            fn()
+        ts = []
+        for _ in range(iters):
+            flush.fill_(0.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return sorted(ts)[len(ts) // 2]
+
+    do = si.make_dout(p.seed + 1, p.B, p.Hq, p.N, p.d).to(q.device)
+    eab.attn_fwd(q, k, v, o, lse, True, p.scale, stream)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    delta = torch.empty_like(lse)
+    t_bwd = timed(lambda: eab.attn_bwd(q, k, v, o, lse, do, delta, dq, dk, dv, True, p.scale, stream))
+    q8, sq = eab.quantize_fp8(q, stream=stream)
+    k8, sk = eab.quantize_fp8(k, stream=stream)
+    vt8, sv = eab.quantize_fp8(v, per_plane=True, transpose=True, stream=stream)
+    o8 = torch.empty_like(o)
+    lse8 = torch.empty_like(lse)
+    t_fp8 = timed(lambda: eab.attn_fwd_fp8(q8, k8, vt8, sq, sk, sv, o8, lse8, True, p.scale, stream))
+    t_quant = timed(lambda: (eab.attn_quant_fp8(q, q8, sq, stream=stream), eab.attn_quant_fp8(k, k8, sk, stream=stream),
+                             eab.attn_quant_fp8(v, vt8, sv, per_plane=True, transpose=True, stream=stream)))
+    torch.cuda.synchronize()
+    assert eab.attn_device_status() == 0
+    return t_bwd, t_fp8, t_quant
+
+
 def run_ours(args):
     import exact_attention_ring_b200 as eab
 
@@ -323,6 +359,27 @@ def run_ours(args):
     dominant = max(times, key=times.get)
     roofline = {"fwd_causal": roof_fwd, "fwd_noncausal": roof_fwd_nc, "decode": roof_dec}[dominant]
 
+    # the backward pass and the FP8 forward, outside the timed step (one GPU only:
+    # no collective runs on this path)
+    extra = None
+    if world == 1:
+        try:
+            t_bwd, t_fp8, t_quant = measure_extra_paths(eab, q, k, v, o, lse, p, flush, stream)
+            fl_bwd = 2.5 * p.flops()  # the five N x N x d products of the backward pass
+            extra = {
+                "note": "timed alone after the step, same prefill workload (causal), L2 flushed, median of 10",
+                "backward": {"ms": round(t_bwd, 5), "tflops": round(fl_bwd / (t_bwd * 1e-3) / 1e12, 1),
+                             "frac_bf16_peak": round(fl_bwd / (t_bwd * 1e-3) / 1e12 / tc_peak, 4),
+                             "launches": "bwd_delta_kernel, bwd_tile_kernel dK/dV, bwd_tile_kernel dQ"},
+                "fp8_forward": {"ms": round(t_fp8, 5), "tflops": round(p.flops() / (t_fp8 * 1e-3) / 1e12, 1),
+                                "peak": round(2 * tc_peak, 1),
+                                "peak_source": "measured bf16_tflops x 2 (nominal fp8 / bf16 ratio)",
+                                "frac": round(p.flops() / (t_fp8 * 1e-3) / 1e12 / (2 * tc_peak), 4),
+                                "quant_ms_q_k_v": round(t_quant, 5)},
+            }
+        except Exception as exc:  # the headline line is printed regardless
+            extra = {"error": f"{type(exc).__name__}: {exc}"}
+
     cpu = cpu_baseline_sample(budget_s=args.cpu_budget) if (rank == 0 and world == 1 and not args.no_cpu) else None
 
     if rank == 0:
@@ -360,6 +417,7 @@ def run_ours(args):
                     "pipeline": "per step: H2D of q,k,v, attn_fwd, D2H of o,lse; copies on their own streams, "
                                 "so step i's kernel overlaps step i+1's input copy and step i-1's output copy"},
             "gpu_launches": 4 * args.steps,
+            "extra_paths": extra,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
             "peaks": {"source": peak_src, "bf16_tflops": tc_peak, "hbm_gbs": hbm_peak},
