@@ -14,19 +14,22 @@
 //   bwd_tile_kernel, DKDV   one 128-key tile of one (batch, KV head) per block:
 //                           for every query head of the group and every query
 //                           tile that sees the keys, S^T = K Q^T and
-//                           dP^T = V dO^T into TMEM, P^T and scale dS^T (bf16)
+//                           dP^T = V dO^T into TMEM, P^T and dS^T (bf16)
 //                           written back over them by the element-wise warps
 //                           (one thread per key), then dV += P^T dO and
-//                           dK += scale dS^T Q with A from TMEM;
+//                           dK += dS^T Q with A from TMEM (scale applied to dK
+//                           once, in the epilogue);
 //   bwd_tile_kernel, !DKDV  one 128-row query tile of one (batch, query head)
 //                           per block: S = Q K^T and dP = dO V^T per key tile,
-//                           scale dS (bf16) over dP, dQ += scale dS K.
+//                           dS (bf16) over dP, dQ += dS K (then times scale).
 // 192 threads each: warps 0-3 element-wise work and epilogue (thread = TMEM
-// lane), warp 4 the MMA issuer, warp 5 the TMA producer. The steps of a block
-// run one after another (the MMAs wait for the element-wise pass and back);
-// the next step's S^T / dP^T MMAs are issued after the accumulating MMAs that
-// read P^T / dS^T from the same columns, so the tensor pipe's issue order keeps
-// them intact until read (as in the forward pass). Every wait is bounded.
+// lane), warp 4 the MMA issuer, warp 5 the TMA producer. Within a step the
+// element-wise pass computes P from S^T while dP^T is still being computed,
+// and hands P and dS over in two halves of 64 columns: the accumulating MMAs
+// of the first half run while the second half is computed. The next step's
+// S^T / dP^T MMAs are issued after the accumulating MMAs that read P^T / dS^T
+// from the same columns, so the tensor pipe's issue order keeps them intact
+// until read (as in the forward pass). Every wait is bounded.
 #pragma once
 
 #include "sm100_ptx.cuh"
