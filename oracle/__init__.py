@@ -54,6 +54,8 @@ def _bind(lib):
     lib.oracle_e4m3_decode.restype = I
     lib.oracle_e4m3_encode.argtypes = [P, L, P]
     lib.oracle_e4m3_encode.restype = I
+    lib.oracle_hadamard_rotate.argtypes = [P, P, L, I, P]
+    lib.oracle_hadamard_rotate.restype = I
     return lib
 
 
@@ -231,3 +233,16 @@ def dequant_fp8(codes, scales):
     N = codes.shape[-2]
     rep = scales.to(torch.float64).repeat_interleave(128, dim=-1)[..., :N]
     return e4m3_decode(codes) * rep.unsqueeze(-1)
+
+
+def hadamard_rotate(x, signs, plant: int = 0):
+    """Incoherent-processing rotation of the rows of x [..., d] (fp32 result):
+    y = H (signs o x) / sqrt(d), H the Sylvester Hadamard matrix, computed as
+    the fast Walsh-Hadamard transform in fp32."""
+    xf = x.to(torch.float32).contiguous()
+    sg = signs.to(torch.float32).contiguous()
+    d = xf.shape[-1]
+    assert sg.shape == (d,)
+    y = torch.empty_like(xf)
+    _check(_load(plant).oracle_hadamard_rotate(_ptr(xf), _ptr(sg), xf.numel() // d, d, _ptr(y)), "hadamard_rotate")
+    return y

@@ -28,6 +28,7 @@
 //  oracle_attention_backward        dQ, dK, dV from the definition
 //  oracle_quant_fp8                 block quantisation to FP8 (E4M3) codes
 //  oracle_e4m3_decode               FP8 (E4M3) code -> value
+//  oracle_hadamard_rotate           the rotation of incoherent processing
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -469,6 +470,38 @@ int oracle_e4m3_decode(const uint8_t* codes, int64_t n, double* out) {
 int oracle_e4m3_encode(const float* x, int64_t n, uint8_t* out) {
     if (x == nullptr || out == nullptr || n < 0) return 1;
     for (int64_t i = 0; i < n; ++i) out[i] = e4m3_code(x[i]);
+    return 0;
+}
+
+// Incoherent processing (FlashAttention-3 page, FP8 with "incoherent
+// processing"; the page gives no detail). Reading taken: each row x of Q and
+// of K is replaced by y = H (sigma o x) / sqrt(d), H the d x d Sylvester
+// Hadamard matrix (H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]]) and sigma a
+// vector of random signs shared by Q and K. H H^T = d I, so the rotation is
+// orthogonal and Q K^T is unchanged, while an outlier in one coordinate is
+// spread over all d of them before quantisation. Computed in fp32 as the fast
+// Walsh-Hadamard transform of the Sylvester recursion (butterflies of span
+// 1, 2, 4, ..., d/2: (a, b) -> (a + b, a - b)), then one multiplication by the
+// fp32 value nearest 1 / sqrt(d).
+//   x, y   [rows, d] fp32 (y written; may equal x)
+//   signs  [d] fp32, each +1 or -1
+int oracle_hadamard_rotate(const float* x, const float* signs, int64_t rows, int d, float* y) {
+    if (x == nullptr || signs == nullptr || y == nullptr || rows < 0 || d < 1 || (d & (d - 1)) != 0) return 1;
+    for (int t = 0; t < d; ++t)
+        if (signs[t] != 1.0f && signs[t] != -1.0f) return 1;
+    const float r = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+    std::vector<float> w(d);
+    for (int64_t i = 0; i < rows; ++i) {
+        for (int t = 0; t < d; ++t) w[t] = signs[t] * x[i * d + t];
+        for (int h = 1; h < d; h *= 2)
+            for (int b = 0; b < d; b += 2 * h)
+                for (int t = b; t < b + h; ++t) {
+                    const float a = w[t], c = w[t + h];
+                    w[t] = a + c;
+                    w[t + h] = a - c;
+                }
+        for (int t = 0; t < d; ++t) y[i * d + t] = (kPlant == 11) ? w[t] : w[t] * r;  // 11: 1/sqrt(d) dropped
+    }
     return 0;
 }
 

@@ -10,8 +10,8 @@ recurrence of the "递归计算softmax" section of "1-Flash-Attention.md").
 The mutation test at the bottom builds oracle variants with one planted
 mistake each (a dropped scale, a wrong GQA grouping, a causal off-by-one, a
 log2 LSE, a missing rescale, a plain-average merge, a transposed K, a dropped
-key, unnormalised partials, E4M3 rounding toward zero) and checks that at
-least one pin fails on each.
+key, unnormalised partials, E4M3 rounding toward zero, a rotation missing its
+1/sqrt(d)) and checks that at least one pin fails on each.
 """
 import math
 
@@ -293,11 +293,34 @@ def pin_quant_fp8_blocks(plant=0):
     assert torch.equal(oracle.quant_fp8(x)[1][1, 2, 1], torch.tensor(1.0))
 
 
+def pin_hadamard_rotation(plant=0):
+    """The incoherent-processing rotation against scipy's Hadamard matrix (within
+    fp32 rounding), its orthogonality (norms and dot products kept, so Q K^T is
+    unchanged), and the exact spreading of a one-hot outlier at d = 64."""
+    import scipy.linalg
+    g = torch.Generator().manual_seed(62)
+    for d in (64, 128):
+        x = torch.randn(40, d, generator=g)
+        z = torch.randn(40, d, generator=g)
+        sg = torch.where(torch.rand(d, generator=g) < 0.5, -1.0, 1.0)
+        y = oracle.hadamard_rotate(x, sg, plant=plant).double()
+        w = oracle.hadamard_rotate(z, sg, plant=plant).double()
+        H = torch.from_numpy(scipy.linalg.hadamard(d)).double()
+        ref = (x.double() * sg.double()) @ H.T / math.sqrt(d)
+        assert (y - ref).abs().max().item() <= 1e-6 * ref.abs().max().item() * math.sqrt(d)
+        assert torch.allclose(y.norm(dim=-1), x.double().norm(dim=-1), rtol=1e-6, atol=0)
+        assert torch.allclose((y * w).sum(-1), (x.double() * z.double()).sum(-1), rtol=0, atol=1e-4)
+    one_hot = torch.zeros(1, 64)
+    one_hot[0, 5] = 100.0
+    y = oracle.hadamard_rotate(one_hot, torch.ones(64), plant=plant)
+    assert torch.equal(y.abs(), torch.full((1, 64), 12.5))
+
+
 PINS = [pin_probs_are_distributions, pin_constant_v, pin_causal_first_row, pin_single_key,
         pin_two_keys_closed_form, pin_identical_keys, pin_library_sdpa, pin_brute_force_tiny,
         pin_blockwise_equals_direct, pin_invariants, pin_decode_and_combine,
         pin_bf16_inputs_widen_exactly, pin_fp16_inputs_widen_exactly, pin_row_sampling,
-        pin_e4m3_codec_matches_torch, pin_quant_fp8_blocks]
+        pin_e4m3_codec_matches_torch, pin_quant_fp8_blocks, pin_hadamard_rotation]
 
 
 def test_backward_matches_autograd():
@@ -345,7 +368,8 @@ def test_pin(pin):
 
 PLANTS = {1: "scale dropped", 2: "GQA head h % Hkv", 3: "causal off by one", 4: "LSE in log2",
           5: "recurrence without rescale", 6: "merge by plain average", 7: "K read transposed",
-          8: "one key dropped", 9: "partials not normalised", 10: "E4M3 rounding toward zero"}
+          8: "one key dropped", 9: "partials not normalised", 10: "E4M3 rounding toward zero",
+          11: "rotation without 1/sqrt(d)"}
 
 
 @pytest.mark.parametrize("plant", sorted(PLANTS), ids=[PLANTS[p] for p in sorted(PLANTS)])
@@ -357,3 +381,33 @@ def test_planted_mistake_is_caught(plant):
         except (AssertionError, ValueError):
             caught.append(pin.__name__)
     assert caught, f"no pin catches planted mistake {plant} ({PLANTS[plant]})"
+
+
+def test_incoherent_processing_lowers_fp8_error():
+    """What the rotation is for (FlashAttention-3 page: FP8 error lowered by
+    incoherent processing): with two outlier channels in Q and K, attention on
+    block-quantised E4M3 inputs is at least twice as close to the exact result
+    when Q and K are rotated first."""
+    import seeded_inputs as si
+    q, k, v = si.make_qkv(11, 1, 2, 2, 256, 128)
+    qf, kf = q.float(), k.float()
+    qf[..., 3] *= 20
+    kf[..., 3] *= 20
+    qf[..., 77] *= 15
+    kf[..., 77] *= 15
+    qf, kf = qf.to(torch.bfloat16), kf.to(torch.bfloat16)
+    sc = 128 ** -0.5
+    o_ref, _ = oracle.attention(qf, kf, v, False, sc)
+    vd = oracle.dequant_fp8(*oracle.quant_fp8(v, per_plane=True))
+    g = torch.Generator().manual_seed(5)
+    sg = torch.where(torch.rand(128, generator=g) < 0.5, -1.0, 1.0)
+
+    def rel_err(qq, kk):
+        qd = oracle.dequant_fp8(*oracle.quant_fp8(qq))
+        kd = oracle.dequant_fp8(*oracle.quant_fp8(kk))
+        o, _ = oracle.attention(qd, kd, vd, False, sc)
+        return ((o - o_ref).pow(2).mean().sqrt() / o_ref.pow(2).mean().sqrt()).item()
+
+    plain = rel_err(qf, kf)
+    rotated = rel_err(oracle.hadamard_rotate(qf, sg), oracle.hadamard_rotate(kf, sg))
+    assert rotated * 2 <= plain, (plain, rotated)
