@@ -1,6 +1,7 @@
-"""Host-side tests of ring attention (context parallelism): the ring schedule
-and the shard exchange over a ring of gloo ranks on the CPU. The attention
-and merge arithmetic run only in the CUDA kernels (tests/test_ring_gpu.py)."""
+"""Host-side tests of ring attention (context parallelism): the ring schedule,
+and ring_attention itself over a ring of gloo ranks on the CPU with its
+per-step attention + merge replaced by a recorder. The attention and merge
+arithmetic run only in the CUDA kernels (tests/test_ring_gpu.py)."""
 import os
 import socket
 
@@ -55,46 +56,58 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _exchange_worker(rank, world, port, causal, q):
+def _ring_worker(rank, world, port, causal, q):
+    """Runs the shipped ring_attention on this gloo rank with the per-step
+    attention + merge replaced by a recorder: the loop, the exchange, the
+    landing buffers and the choice of the step that writes O are the product's
+    own code."""
     import sys
     sys.path.insert(0, ROOT)
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        from exact_attention_ring_b200.ring import ring_exchange, ring_schedule
-        # this rank's "shards": tensors that identify their owner in every element
-        k = torch.full((2, 3, 5, 4), float(rank))
-        v = torch.full((2, 1, 5, 4), 100.0 + rank)
-        landing = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(min(2, world - 1))]
-        cur, held = (k, v), []
-        for s, (src, _) in enumerate(ring_schedule(rank, world, causal)):
-            reqs = []
-            if s + 1 < world:
-                nxt = landing[s % 2]
-                reqs = ring_exchange(list(cur), list(nxt))
-            held.append((src, bool(torch.all(cur[0] == src)), bool(torch.all(cur[1] == 100.0 + src))))
-            for r in reqs:
-                r.wait()
-            if s + 1 < world:
-                cur = nxt
-        q.put((rank, held, bool(torch.all(k == rank)), bool(torch.all(v == 100.0 + rank))))
+        import exact_attention_ring_b200.ring as ring
+        calls = []
+
+        def record(self, k, v, kind, out=None, stream=None):
+            # the key/value shard this step holds is identified by its contents
+            k0, v0 = float(k.flatten()[0]), float(v.flatten()[0])
+            calls.append((k0, bool(torch.all(k == k0)), v0, bool(torch.all(v == v0)), kind, out is not None))
+
+        ring._RankState.add = record
+        qs = torch.zeros(2, 4, 5, 8, dtype=torch.bfloat16)
+        k = torch.full((2, 2, 5, 8), float(rank), dtype=torch.bfloat16)
+        v = torch.full((2, 2, 5, 8), 100.0 + rank, dtype=torch.bfloat16)
+        o, lse = ring.ring_attention(qs, k, v, causal=causal)
+        q.put((rank, calls, bool(torch.all(k == rank)), bool(torch.all(v == 100.0 + rank)),
+               tuple(o.shape), tuple(lse.shape)))
     finally:
         dist.destroy_process_group()
 
 
 @pytest.mark.parametrize("world", [2, 3])
-def test_ring_exchange_moves_shards_around_the_ring(world):
-    """Every rank holds, in step s, exactly the shard the schedule names; its own
-    inputs are left untouched."""
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_attention_steps_on_gloo_ranks(world, causal):
+    """ring_attention itself, on a ring of gloo ranks: in step s every rank holds
+    exactly the shard the schedule names (with its kind), the last step that is
+    not skipped alone writes O, and the caller's K and V are left untouched."""
+    ring_schedule, FULL, DIAG, SKIP = _schedule()
     ctx = mp.get_context("spawn")
     q = ctx.SimpleQueue()
-    mp.start_processes(_exchange_worker, args=(world, _free_port(), True, q), nprocs=world, join=True,
+    mp.start_processes(_ring_worker, args=(world, _free_port(), causal, q), nprocs=world, join=True,
                        start_method="spawn")
     results = sorted(q.get() for _ in range(world))
-    for rank, held, k_intact, v_intact in results:
+    assert [r[0] for r in results] == list(range(world))
+    for rank, calls, k_intact, v_intact, o_shape, lse_shape in results:
         assert k_intact and v_intact
-        assert [src for src, _, _ in held] == [(rank - s) % world for s in range(world)]
-        assert all(kok and vok for _, kok, vok in held), held
+        assert o_shape == (2, 4, 5, 8) and lse_shape == (2, 4, 5)
+        sched = ring_schedule(rank, world, causal)
+        assert len(calls) == world
+        for (k0, k_uni, v0, v_uni, kind, wrote), (src, skind) in zip(calls, sched):
+            assert k_uni and v_uni
+            assert (k0, v0, kind) == (float(src), 100.0 + src, skind)
+        last = max(s for s, (_, kind) in enumerate(sched) if kind != SKIP)
+        assert [wrote for *_, wrote in calls] == [s == last for s in range(world)]
 
 
 def test_ring_compute_has_no_cpu_path():
