@@ -20,6 +20,12 @@ elapsed time is the max over ranks.
 
 --impl reference times the float64 CPU oracle (the checker) on the host cores
 on a bounded sample of the same causal prefill workload; rank 0 only.
+
+    python bench.py profile fwd|decode|merge|ring|bwd [--B ..] [--H ..] ...
+
+runs one kernel of the library a few times on seeded inputs (no timing loop,
+no oracle) and prints the CUDA-event time of the last launch: the command that
+the ncu captures under profiles/ wrap.
 """
 from __future__ import annotations
 
@@ -430,64 +436,165 @@ def run_ours(args):
 
 # ------------------------------------------------------------ oracle timing --
 
-def _oracle_slices(n_slices, budget_s, seed_offset=0):
-    """Times the oracle on whole (b, h) slices of the causal prefill, stopping
-    after `budget_s` seconds or `n_slices` slices. Returns (flops, seconds, k)."""
-    import oracle
-    p = PREFILL
-    q, k, v = si.make_qkv(p.seed + seed_offset, p.B, p.Hq, p.Hkv, p.N, p.d)
-    per_slice = 4.0 * p.N * (p.N + 1) / 2 * p.d  # causal: row i sees i+1 keys
-    done, elapsed = 0, 0.0
-    order = torch.randperm(p.B * p.Hq, generator=torch.Generator().manual_seed(5)).tolist()
-    for s in order[:n_slices]:
-        rows = torch.arange(s * p.N, (s + 1) * p.N, dtype=torch.int64)
-        t0 = time.perf_counter()
-        oracle.attention(q, k, v, True, p.scale, rows=rows)
-        elapsed += time.perf_counter() - t0
-        done += 1
-        if elapsed >= budget_s:
-            break
-    return done * per_slice, elapsed, done
+class OracleSampler:
+    """Times the float64 oracle on whole (b, h) slices of the causal prefill
+    workload (same seeded inputs as the GPU arm, drawn once), walking a fixed
+    random order of the slices. The CPU baseline of our arm and the reference
+    arm both time through this one sampler, so their figures are the same
+    measurement (per-slice work is identical: every slice is 2048 causal rows)."""
+
+    SLICES_PER_STEP = 4  # reference arm: slices timed per step
+
+    def __init__(self):
+        import oracle
+        self.oracle = oracle
+        p = PREFILL
+        self.q, self.k, self.v = si.make_qkv(p.seed, p.B, p.Hq, p.Hkv, p.N, p.d)
+        self.per_slice = 4.0 * p.N * (p.N + 1) / 2 * p.d  # causal: row i sees i+1 keys
+        self.order = torch.randperm(p.B * p.Hq, generator=torch.Generator().manual_seed(5)).tolist()
+        self.next = 0
+
+    def time(self, n_slices, budget_s=float("inf")):
+        """(flops, seconds, slices) for the next `n_slices` slices, stopping early
+        once `budget_s` seconds of oracle time have been spent."""
+        p = PREFILL
+        done, elapsed = 0, 0.0
+        while done < n_slices and elapsed < budget_s:
+            sl = self.order[self.next % len(self.order)]
+            self.next += 1
+            rows = torch.arange(sl * p.N, (sl + 1) * p.N, dtype=torch.int64)
+            t0 = time.perf_counter()
+            self.oracle.attention(self.q, self.k, self.v, True, p.scale, rows=rows)
+            elapsed += time.perf_counter() - t0
+            done += 1
+        return done * self.per_slice, elapsed, done
 
 
 def cpu_baseline_sample(budget_s=15.0):
-    import oracle
-    flops, secs, k = _oracle_slices(PREFILL.B * PREFILL.Hq, budget_s)
-    return {"value": flops / secs / 1e12, "unit": "TFLOPS", "cores": oracle.hardware_threads(), "kind": "oracle",
+    smp = OracleSampler()
+    smp.time(1)  # warm-up: thread pool and first-touch pages
+    flops, secs, k = smp.time(PREFILL.B * PREFILL.Hq, budget_s)
+    return {"value": flops / secs / 1e12, "unit": "TFLOPS", "cores": smp.oracle.hardware_threads(), "kind": "oracle",
             "sample": f"{k} of {PREFILL.B * PREFILL.Hq} (b,h) slices of the causal prefill B2 H32 N2048 d128, all "
-                      f"2048 rows each ({secs:.1f} s of float64 CPU work, all host threads)"}
+                      f"2048 rows each ({secs:.1f} s of float64 CPU work, all host threads), after one warm-up slice"}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    import oracle
     p = PREFILL
+    smp = OracleSampler()
     for _ in range(args.warmup):
-        _oracle_slices(1, 0.0)
+        smp.time(1)
     flops, secs = 0.0, 0.0
-    for i in range(args.steps):
-        f, s, _ = _oracle_slices(1, 0.0, seed_offset=0)
+    for _ in range(args.steps):
+        f, sec, _ = smp.time(OracleSampler.SLICES_PER_STEP)
         flops += f
-        secs += s
+        secs += sec
     val = flops / secs / 1e12
-    cores = oracle.hardware_threads()
+    cores = smp.oracle.hardware_threads()
+    k = OracleSampler.SLICES_PER_STEP
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1), bf16 widened to f64)",
-        "config": {"workload": "prefill B2 H32 N2048 d128 causal (LLaMA-7B shape); one (b,h) slice per step",
+        "config": {"workload": f"prefill B2 H32 N2048 d128 causal (LLaMA-7B shape); {k} (b,h) slices per step",
                    "prefill": {"B": p.B, "Hq": p.Hq, "Hkv": p.Hkv, "N": p.N, "d": p.d, "causal": True}},
         "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
-                         "sample": "one (b,h) slice (2048 rows) of the causal prefill per step"},
+                         "sample": f"{k} (b,h) slices (2048 causal rows each) of the causal prefill per step, "
+                                   f"the same slice sampler as our arm's cpu_baseline"},
         "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------- profile cases --
+
+def run_profile_case(argv):
+    """One kernel of the library a few times on seeded inputs, for profilers
+    (one kernel, a few launches, inputs larger than L2 but a few GB at most)."""
+    import exact_attention_ring_b200 as eab
+    ap = argparse.ArgumentParser(prog="bench.py profile")
+    ap.add_argument("kernel", choices=["fwd", "decode", "merge", "ring", "bwd", "fp8"])
+    ap.add_argument("--B", type=int, default=4)
+    ap.add_argument("--H", type=int, default=32)
+    ap.add_argument("--Hkv", type=int, default=0)
+    ap.add_argument("--N", type=int, default=2048)
+    ap.add_argument("--L", type=int, default=131072)
+    ap.add_argument("--d", type=int, default=128)
+    ap.add_argument("--causal", type=int, default=1)
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--world", type=int, default=4, help="ring: virtual ranks emulated on this GPU")
+    a = ap.parse_args(argv)
+    Hkv = a.Hkv or a.H
+    dev = torch.device("cuda", 0)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    scale = a.d ** -0.5
+    if a.kernel in ("fwd", "bwd", "ring", "fp8"):
+        q, k, v = (t.to(dev) for t in si.make_qkv(1001, a.B, a.H, Hkv, a.N, a.d))
+    if a.kernel == "fwd":
+        o = torch.empty_like(q)
+        lse = torch.empty(a.B, a.H, a.N, device=dev)
+        fn = lambda: eab.attn_fwd(q, k, v, o, lse, bool(a.causal), scale)  # noqa: E731
+        work = 4.0 * a.B * a.H * a.N * a.N * a.d / (2 if a.causal else 1)
+    elif a.kernel == "fp8":
+        # the forward on E4M3 codes (the three quantisations run once, before)
+        q8, sq = eab.quantize_fp8(q)
+        k8, sk = eab.quantize_fp8(k)
+        vt8, sv = eab.quantize_fp8(v, per_plane=True, transpose=True)
+        o = torch.empty_like(q)
+        lse = torch.empty(a.B, a.H, a.N, device=dev)
+        fn = lambda: eab.attn_fwd_fp8(q8, k8, vt8, sq, sk, sv, o, lse, bool(a.causal), scale)  # noqa: E731
+        work = 4.0 * a.B * a.H * a.N * a.N * a.d / (2 if a.causal else 1)
+    elif a.kernel == "merge":
+        # one merge step of a ring: fp32 accumulator read and written, fp32 block
+        # and the two LSE vectors read
+        rows = a.B * a.H * a.N
+        g = torch.Generator().manual_seed(1005)
+        o_acc = torch.randn(rows, a.d, generator=g).to(dev)
+        lse_acc = torch.randn(rows, generator=g).to(dev)
+        o_blk = torch.randn(rows, a.d, generator=g).to(dev)
+        lse_blk = torch.randn(rows, generator=g).to(dev)
+        fn = lambda: eab.attn_merge(o_acc, lse_acc, o_blk, lse_blk)  # noqa: E731
+        work = rows * (a.d * (4 + 4 + 4) + 4 * 3)
+    elif a.kernel == "bwd":
+        # the three launches of attn_bwd (Delta, dK/dV, dQ) on the forward's O, LSE;
+        # FLOPs counted as the five N x N x d products of the backward pass
+        do = si.make_dout(1002, a.B, a.H, a.N, a.d).to(dev)
+        o, lse = eab.attention(q, k, v, bool(a.causal), scale)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        delta = torch.empty_like(lse)
+        fn = lambda: eab.attn_bwd(q, k, v, o, lse, do, delta, dq, dk, dv, bool(a.causal), scale)  # noqa: E731
+        work = 10.0 * a.B * a.H * a.N * a.N * a.d / (2 if a.causal else 1)
+    elif a.kernel == "ring":
+        # every virtual rank's steps of the ring, one after another on this GPU
+        fn = lambda: eab.ring_attention_emulated(q, k, v, a.world, bool(a.causal), scale)  # noqa: E731
+        work = 4.0 * a.B * a.H * a.N * a.N * a.d / (2 if a.causal else 1)
+    else:
+        qd, kd, vd = (t.to(dev) for t in si.make_decode(1004, a.B, a.H, Hkv, a.L, a.d))
+        S = eab.attn_decode_default_splits(a.B, a.H, Hkv, a.L)
+        o_part = torch.empty(a.B, a.H, S, a.d, device=dev)
+        lse_part = torch.empty(a.B, a.H, S, device=dev)
+        fn = lambda: eab.attn_decode_splitkv(qd, kd, vd, o_part, lse_part, S, scale)  # noqa: E731
+        work = 2.0 * a.B * Hkv * a.L * a.d * 2
+    for _ in range(a.iters):
+        start.record()
+        fn()
+        end.record()
+    torch.cuda.synchronize()
+    assert eab.attn_device_status() == 0
+    ms = start.elapsed_time(end)
+    tensor = a.kernel in ("fwd", "ring", "bwd", "fp8")
+    print(f"{a.kernel}: {ms:.4f} ms  {work / (ms * 1e-3) / (1e12 if tensor else 1e9):.1f} "
+          f"{'TFLOPS' if tensor else 'GB/s'}")
+
+
 def main():
+    if len(sys.argv) > 1 and sys.argv[1] == "profile":
+        run_profile_case(sys.argv[2:])
+        return
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
