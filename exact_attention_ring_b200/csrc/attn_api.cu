@@ -80,6 +80,10 @@ bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// The combine keeps one weight per split in dynamic shared memory; with its few
+// static words it must stay under the 48 KiB a launch gets without opting in.
+constexpr int kCombineMaxSplits = 12000;
+
 template <int D, bool CAUSAL, bool F32OUT, class E>
 attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                          cudaStream_t stream) {
@@ -104,6 +108,20 @@ attn_status_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const 
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
     const dim3 grid(p.S, p.Hkv * p.groups, p.B);
+    kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+constexpr int kDecodeKeysSlots = 3;  // K/V ring of the keys-as-rows decode (3 slots: two blocks per SM)
+
+template <int NQ, class E>
+attn_status_t launch_decode_keys(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                                 cudaStream_t stream) {
+    using C = DecTCfg<NQ, kDecodeKeysSlots>;
+    auto kern = decode_splitkv_keys_kernel<NQ, kDecodeKeysSlots, E>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    const dim3 grid(p.S, p.Hkv, p.B);
     kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -195,6 +213,10 @@ attn_status_t decode_impl(const void* q, const void* k, const void* v, float* o_
     if (static_cast<long long>(Hkv) * p.groups > 65535) return ATTN_ERR_INVALID_ARG;
     p.scale_log2 = scale * kLog2e;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // small groups at d = 128: keys as the tile rows (a few query heads cannot
+    // fill 128 rows); other shapes: the query heads as the tile rows
+    if (d == 128 && p.G <= 16) return launch_decode_keys<16, E>(tk, tv, p, st);
+    if (d == 128 && p.G <= 32) return launch_decode_keys<32, E>(tk, tv, p, st);
     return d == 128 ? launch_decode<128, E>(tk, tv, p, st) : launch_decode<64, E>(tk, tv, p, st);
 }
 
@@ -206,7 +228,7 @@ attn_status_t combine_impl(const float* o_part, const float* lse_part, void* o, 
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     const long long blocks = static_cast<long long>(B) * Hq;
     const size_t smem = static_cast<size_t>(num_splits) * sizeof(float);
-    if (blocks > 0x7fffffffLL || smem > 48 * 1024) return ATTN_ERR_INVALID_ARG;
+    if (blocks > 0x7fffffffLL || num_splits > kCombineMaxSplits) return ATTN_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     auto* ob = static_cast<typename E::T*>(o);
     if (d == 128)
@@ -327,13 +349,19 @@ attn_status_t attn_quant_fp8(const void* x, void* codes, float* scales, int plan
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     const int nblk = (N + 127) / 128;
     if (planes > 65535) return ATTN_ERR_INVALID_ARG;
-    QuantParams p;
+    QuantParams p{};
     p.x = static_cast<const __nv_bfloat16*>(x);
     p.codes = static_cast<uint8_t*>(codes);
     p.scales = scales;
     p.planes = planes; p.N = N; p.nblk = nblk; p.Np = nblk * 128; p.per_plane = per_plane;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const dim3 grid(nblk, planes);
+    if (!per_plane && !transpose) {
+        // per-block scales, row-major codes: one pass over x
+        if (d == 128) fp8_quant_rows_kernel<128, false><<<grid, 256, 0, st>>>(p);
+        else fp8_quant_rows_kernel<64, false><<<grid, 256, 0, st>>>(p);
+        return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    }
     if (d == 128) {
         fp8_amax_kernel<128><<<grid, 256, 0, st>>>(p);
         if (transpose) fp8_quant_kernel<128, true><<<grid, 256, 0, st>>>(p);
@@ -344,6 +372,26 @@ attn_status_t attn_quant_fp8(const void* x, void* codes, float* scales, int plan
         else fp8_quant_kernel<64, false><<<grid, 256, 0, st>>>(p);
     }
     fp8_scales_kernel<<<(planes + 255) / 256, 256, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_quant_fp8_rotate(const void* x, const float* signs, void* codes, float* scales, int planes, int N,
+                                    int d, attn_stream_t stream) {
+    if (!aligned16(x) || !aligned16(signs) || !aligned16(codes) || !aligned16(scales)) return ATTN_ERR_INVALID_ARG;
+    if (planes < 1 || N < 1 || planes > 65535) return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    const int nblk = (N + 127) / 128;
+    QuantParams p{};
+    p.x = static_cast<const __nv_bfloat16*>(x);
+    p.codes = static_cast<uint8_t*>(codes);
+    p.scales = scales;
+    p.planes = planes; p.N = N; p.nblk = nblk; p.Np = nblk * 128; p.per_plane = 0;
+    p.signs = signs;
+    p.rot_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid(nblk, planes);
+    if (d == 128) fp8_quant_rows_kernel<128, true><<<grid, 256, 0, st>>>(p);
+    else fp8_quant_rows_kernel<64, true><<<grid, 256, 0, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -378,13 +426,15 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, cons
 
 int attn_decode_default_splits(int B, int Hq, int Hkv, int L) {
     if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0) return 0;
-    // One decode block runs per SM (148 on B200) and streams its split at about
-    // the SM's share of HBM bandwidth after a fixed start-up worth ~260 keys.
-    // Pick the split count that maximises (busy fraction of the SM waves) x
-    // (streaming fraction chunk / (chunk + 260)); splits are whole 128-key tiles.
-    constexpr int kSMs = 148, kStage = 128;
-    constexpr double kStartupKeys = 260.0;
+    // Decode blocks (one per SM, 148 on B200; two per SM for the keys-as-rows
+    // kernel with a 3-slot ring) each stream their split at about their share of
+    // HBM bandwidth after a fixed start-up worth ~260 keys. Pick the split count
+    // that maximises (busy fraction of the block waves) x (streaming fraction
+    // chunk / (chunk + 260)); splits are whole 128-key tiles.
     const int G = Hq / Hkv;
+    const int kSMs = 148 * (G <= 32 ? DecTCfg<16, kDecodeKeysSlots>::BLOCKS_PER_SM : 1);
+    constexpr int kStage = 128;
+    constexpr double kStartupKeys = 260.0;
     const long long units = static_cast<long long>(B) * Hkv * ((G + 127) / 128);
     const int max_s = static_cast<int>(std::min<long long>((L + kStage - 1) / kStage, 4096));
     int best_s = 1;
@@ -466,6 +516,11 @@ extern "C" attn_status_t attn_decode_noalloc(const void* q, const void* k, const
         return ATTN_ERR_INVALID_ARG;
     if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || num_splits < 1 || num_splits > L) return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    // every limit of the two launches is checked here, so that nothing is
+    // enqueued unless both can run
+    if (num_splits > kCombineMaxSplits || Hq % Hkv != 0 || !scale_ok(scale) || B > 65535 ||
+        static_cast<long long>(Hkv) * ((Hq / Hkv + 127) / 128) > 65535)
+        return ATTN_ERR_INVALID_ARG;
     // partials: o_part [B,Hq,S,d] then lse_part [B,Hq,S], all fp32
     const unsigned long long units = static_cast<unsigned long long>(B) * Hq * num_splits;
     if (units * (static_cast<unsigned long long>(d) + 1) > kNoAllocScratchFloats) return ATTN_ERR_INVALID_ARG;

@@ -324,6 +324,358 @@ __global__ void __launch_bounds__(224, 1)
                     }
                 }
                 if (real) p.lse_part[out_row * p.S + split] = (m_used + log2f(l)) * 0.69314718055994530942f;
+            } else if (real) {
+                // a wait was abandoned (timeout, recorded in the status word): leave an
+                // empty partial (zero weight in the combine) rather than stale memory
+                float* dst = p.o_part + (out_row * p.S + split) * D;
+                for (int c = 0; c < D; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+                p.lse_part[out_row * p.S + split] = -INFINITY;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------- decode, keys as tile rows ----
+// The same split-KV partials for a small group (G = Hq / Hkv <= 32 query heads
+// per key/value head, d = 128), computed transposed so that the 128 keys of a
+// tile, not the few query heads, fill the 128 rows of the tensor-core tile:
+//   S^T = K_j Q^T    tcgen05.mma, A = K_j (128 keys x d, K-major, as TMA lands
+//                    it), B = the group's queries (NQ = 16 or 32 rows, zeros past
+//                    G) -> TMEM, 128 lanes (keys) x NQ columns;
+//   softmax          thread t owns key t of the tile: its NQ scores, per query
+//                    column a maximum over the 128 keys (warp shuffles, then the
+//                    four warps through shared memory), the lazy rescale
+//                    (threshold 2^8, log2 units), NQ exponentials per thread
+//                    instead of 128, a per-thread partial sum of p per column;
+//                    P (bf16) goes to shared memory as a K-major operand;
+//   O^T += V_j^T P   tcgen05.mma, A = V_j read MN-major (the head dimension is
+//                    contiguous), B = P -> TMEM, 128 lanes (head dim) x NQ.
+// The exp2 work per tile drops from 128 x 128 to 128 x NQ, so a block streams
+// K and V at the rate TMA and HBM deliver, and TMEM use drops to 64 or 128
+// columns. Warp roles and the K_0 K_1 V_0 K_2 V_1 ... load order are those of
+// decode_splitkv_kernel. TMEM columns: S^T buffers [0, NQ), [NQ, 2 NQ), O^T
+// [2 NQ, 3 NQ).
+template <int NQ, int SLOTS_ = 6>
+struct DecTCfg {
+    static constexpr int D = 128, BN = 128, CHUNKS = D / 64;
+    static constexpr int Q_BYTES = CHUNKS * NQ * 128;  // queries as the B operand, [chunk][NQ rows][128 B]
+    static constexpr int P_BYTES = 2 * NQ * 128;       // P as the B operand, [key chunk][NQ rows][128 B]
+    static constexpr int TILE_BYTES = BN * D * 2;
+    static constexpr int SLOTS = SLOTS_;
+    static constexpr int NUM_THREADS = 224;
+    static constexpr int BLOCKS_PER_SM = SLOTS <= 3 ? 2 : 1;  // shared memory: 6 slots take a whole SM
+    static constexpr int RED_FLOATS = 3 * 4 * NQ;      // column maxima (two buffers) and sums of the four warps
+    // q_ready, slot_full, slot_empty, s_full[2], p_full[2], o_done[2], drain, red_bar[2], sum_bar
+    static constexpr int NUM_BARRIERS = 1 + 2 * SLOTS + 2 + 2 + 2 + 1 + 2 + 1;
+    static constexpr int SMEM_BYTES =
+        1024 + Q_BYTES + 2 * P_BYTES + SLOTS * TILE_BYTES + RED_FLOATS * 4 + NUM_BARRIERS * 8 + 16;
+    static constexpr uint32_t TMEM_COLS = NQ <= 16 ? 64 : 128;
+    static constexpr float RESCALE_THRESHOLD = 8.0f;
+};
+
+template <int NQ>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NQ]) {
+    if constexpr (NQ == 16) tmem_ld16(taddr, r);
+    else tmem_ld32(taddr, r);
+}
+template <int NQ>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[NQ]) {
+    if constexpr (NQ == 16) tmem_st16(taddr, r);
+    else tmem_st32(taddr, r);
+}
+
+template <int NQ, int SLOTS_, class E>
+__global__ void __launch_bounds__(224, DecTCfg<NQ, SLOTS_>::BLOCKS_PER_SM)
+    decode_splitkv_keys_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                               const DecodeParams p) {
+    using C = DecTCfg<NQ, SLOTS_>;
+    constexpr int D = C::D, BN = C::BN, SLOTS = C::SLOTS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = smem;
+    uint8_t* sP = sQ + C::Q_BYTES;                 // two P buffers
+    uint8_t* sKV = sP + 2 * C::P_BYTES;
+    float* red = reinterpret_cast<float*>(sKV + SLOTS * C::TILE_BYTES);  // [3][4][NQ]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(red + C::RED_FLOATS);
+    uint64_t* q_ready = bars;                  // queries staged (one arrival per warp 0-3)
+    uint64_t* slot_full = q_ready + 1;         // [SLOTS]
+    uint64_t* slot_empty = slot_full + SLOTS;  // [SLOTS]
+    uint64_t* s_full = slot_empty + SLOTS;     // [2]
+    uint64_t* p_full = s_full + 2;             // [2] (one arrival per softmax warp)
+    uint64_t* o_done = p_full + 2;             // [2] P V(j) completes phase j >> 1 of o_done[j & 1]
+    uint64_t* drain = o_done + 2;
+    uint64_t* red_bar = drain + 1;             // [2] the four softmax warps' column maxima of a tile
+    uint64_t* sum_bar = red_bar + 2;           // the four softmax warps' column sums
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sum_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int G = p.G;                                    // query heads of this group (<= NQ)
+    const size_t row0 = static_cast<size_t>(b) * p.Hq + static_cast<size_t>(hk) * G;  // first output row
+    const int k0 = split * p.chunk;
+    const int k1 = min(p.L, k0 + p.chunk);
+    const int nt = k1 > k0 ? (k1 - k0 + BN - 1) / BN : 0;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_ready, 4);
+        for (int i = 0; i < SLOTS; ++i) {
+            mbar_init(&slot_full[i], C::CHUNKS);
+            mbar_init(&slot_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 4);
+            mbar_init(&o_done[i], 1);
+        }
+        mbar_init(drain, 1);
+        mbar_init(&red_bar[0], 4);
+        mbar_init(&red_bar[1], 4);
+        mbar_init(sum_bar, 4);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 4) {
+        tmem_alloc(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp >= 5) {
+        // ------------------------------------------------------ producers ---
+        if (lane == 0 && nt > 0) {
+            const int me = warp - 5;
+            constexpr uint32_t BOX_BYTES = BN * 128;
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            const int z = b * p.Hkv + hk;
+            int issued = 0;
+            for (int i = 0; i < 2 * nt; ++i) {
+                bool mine = false;
+#pragma unroll
+                for (int c = 0; c < C::CHUNKS; ++c) mine |= ((i * C::CHUNKS + c) & 1) == me;
+                if (!mine) continue;
+                const int slot = i % SLOTS, use = i / SLOTS;
+                if (use > 0 && !mbar_wait(&slot_empty[slot], (use - 1) & 1, abort_flag)) break;
+                int j;
+                const CUtensorMap* tm = dec_load_kind(i, nt, &j) ? &tm_v : &tm_k;
+                uint8_t* dst = sKV + slot * C::TILE_BYTES;
+#pragma unroll
+                for (int c = 0; c < C::CHUNKS; ++c) {
+                    if (((i * C::CHUNKS + c) & 1) != me) continue;
+                    mbar_arrive_expect_tx(&slot_full[slot], BOX_BYTES);
+                    tma_load_3d(dst + c * BOX_BYTES, tm, &slot_full[slot], c * 64, k0 + j * BN, z);
+                }
+                issued = i + 1;
+            }
+            // Let every copy in flight land before the CTA can exit.
+            for (int i = max(0, issued - SLOTS); i < issued; ++i)
+                mbar_wait(&slot_full[i % SLOTS], (i / SLOTS) & 1, nullptr);
+        }
+    } else if (warp == 4) {
+        // ---------------------------------------------------- MMA issuer ----
+        if (lane == 0 && nt > 0) {
+            constexpr uint32_t idesc_s = make_idesc(BN, NQ, 0, 0, E::fmt);  // M = keys, N = queries
+            constexpr uint32_t idesc_o = make_idesc(D, NQ, 1, 0, E::fmt);   // M = head dim (V read MN-major)
+            const uint32_t o_tmem = tmem + 2 * NQ;
+            const uint32_t q_addr = smem_addr(sQ), p_addr = smem_addr(sP), kv_addr = smem_addr(sKV);
+            bool ok = mbar_wait(q_ready, 0, abort_flag);
+            auto issue_s = [&](int j) -> bool {
+                const int ik = dec_kpos(j);
+                if (!mbar_wait(&slot_full[ik % SLOTS], (ik / SLOTS) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t k_addr = kv_addr + (ik % SLOTS) * C::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk & 3) * 32;
+                    const uint64_t ad = make_sdesc_sw128(k_addr + (kk >> 2) * (BN * 128) + koff, 16, 1024);
+                    const uint64_t bd = make_sdesc_sw128(q_addr + (kk >> 2) * (NQ * 128) + koff, 16, 1024);
+                    mma_ss(tmem + (j & 1) * NQ, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(&s_full[j & 1]);
+                tc_commit(&slot_empty[ik % SLOTS]);
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            if (ok && nt > 1) ok = issue_s(1);
+            for (int j = 0; ok && j < nt; ++j) {
+                // O^T += V_j^T P(j), then S^T(j+2) into the S buffer P(j) came from
+                const int iv = dec_vpos(j, nt);
+                ok = mbar_wait(&slot_full[iv % SLOTS], (iv / SLOTS) & 1, abort_flag) &&
+                     mbar_wait_spin(&p_full[j & 1], (j >> 1) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t v_addr = kv_addr + (iv % SLOTS) * C::TILE_BYTES;
+                const uint32_t pb = p_addr + (j & 1) * C::P_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    // 16 keys per step: rows kk*16.. of the V tile (MN-major A, the
+                    // head dimension's two 64-column chunks BN * 128 bytes apart), and
+                    // 32 bytes of every P row (K-major B)
+                    const uint64_t ad = make_sdesc_sw128(v_addr + kk * 16 * 128, BN * 128, 1024);
+                    const uint64_t bd = make_sdesc_sw128(pb + (kk >> 2) * (NQ * 128) + (kk & 3) * 32, 16, 1024);
+                    mma_ss(o_tmem, ad, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(&o_done[j & 1]);
+                tc_commit(&slot_empty[iv % SLOTS]);
+                if (j + 2 < nt) ok = issue_s(j + 2);
+            }
+            // Every MMA must be complete before TMEM is released.
+            tc_commit(drain);
+            mbar_wait(drain, 0, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------- query staging, softmax ----
+        const int t = threadIdx.x;  // key t of each tile; lane t of S^T and of O^T (head-dim element t)
+        if (nt > 0) {
+            // the group's queries as NQ rows of the K-major 128-byte-swizzled operand
+            // (rows past G as zeros): 16-byte unit u of row r of chunk c sits at
+            // unit u ^ (r & 7)
+            for (int i = t; i < NQ * (D / 8); i += 128) {
+                const int r = i / (D / 8), u = i % (D / 8);
+                uint4 v4 = make_uint4(0u, 0u, 0u, 0u);
+                if (r < G) v4 = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.q) + (row0 + r) * D + u * 8);
+                *reinterpret_cast<uint4*>(sQ + (u >> 3) * (NQ * 128) + r * 128 + (((u & 7) ^ (r & 7)) << 4)) = v4;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_ready);
+        }
+        if (nt == 0) {
+            // an empty split: weight 0 in the combine
+            for (int c = 0; c < G; ++c) p.o_part[((row0 + c) * p.S + split) * D + t] = 0.f;
+            if (t < G) p.lse_part[(row0 + t) * p.S + split] = -INFINITY;
+        } else {
+            const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
+            const uint32_t o_addr = lane_base + 2 * NQ;
+            const float c2 = p.scale_log2;
+            float m_used[NQ], lsum[NQ];
+#pragma unroll
+            for (int c = 0; c < NQ; ++c) {
+                m_used[c] = -INFINITY;
+                lsum[c] = 0.f;
+            }
+            bool ok = true;
+            for (int j = 0; j < nt; ++j) {
+                const bool w1 = mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag);
+                if (!__all_sync(0xffffffffu, w1)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t sv[NQ];
+                tmem_ld_cols<NQ>(lane_base + (j & 1) * NQ, sv);
+                const bool valid = k0 + j * BN + t < k1;
+                float s2[NQ];
+#pragma unroll
+                for (int c = 0; c < NQ; ++c) s2[c] = valid ? __uint_as_float(sv[c]) * c2 : -INFINITY;
+                // per query column: maximum over the tile's 128 keys
+                float* rmax = red + (j & 1) * 4 * NQ;
+#pragma unroll
+                for (int c = 0; c < NQ; ++c) {
+                    if (c < G) {
+                        float m = s2[c];
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+                        if (lane == 0) rmax[warp * NQ + c] = m;
+                    }
+                }
+                // exchange through an mbarrier (a bounded wait: no warp can hang the
+                // others if one gives up); tile j completes phase j >> 1 of
+                // red_bar[j & 1], and no warp arrives for tile j + 2 before every warp
+                // has passed tile j + 1
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&red_bar[j & 1]);
+                const bool w2 = mbar_wait(&red_bar[j & 1], (j >> 1) & 1, abort_flag);
+                if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
+                bool any = false;
+                float factor[NQ];
+#pragma unroll
+                for (int c = 0; c < NQ; ++c) {
+                    factor[c] = 1.f;
+                    if (c < G) {
+                        const float mt = fmaxf(fmaxf(rmax[c], rmax[NQ + c]), fmaxf(rmax[2 * NQ + c], rmax[3 * NQ + c]));
+                        if (mt > m_used[c] + C::RESCALE_THRESHOLD) {
+                            factor[c] = ex2_approx(m_used[c] - mt);
+                            m_used[c] = mt;
+                            any = true;
+                        }
+                    }
+                    lsum[c] *= factor[c];
+                }
+                // every thread of the four warps takes the same decision (the maxima are shared)
+                if (j > 0 && any) {
+                    // O^T must hold P V(j-1) before it is rescaled (S(j) implies only P V(j-2))
+                    const bool w3 = mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag);
+                    if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
+                    tc_fence_after();
+                    uint32_t ov[NQ];
+                    tmem_ld_cols<NQ>(o_addr, ov);
+#pragma unroll
+                    for (int c = 0; c < NQ; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * factor[c]);
+                    tmem_st_cols<NQ>(o_addr, ov);
+                    tmem_st_wait();
+                }
+                // P(j): p = exp2(s * c2 - m) for the real columns, into the P buffer
+                // of this parity (P V(j-2), its last reader, is complete: S(j) is)
+                uint8_t* pb = sP + (j & 1) * C::P_BYTES + (t >> 6) * (NQ * 128) + (t & 7) * 2;
+                const int unit = (t & 63) >> 3;
+#pragma unroll
+                for (int c = 0; c < NQ; ++c) {
+                    float pv = 0.f;
+                    if (c < G) {
+                        pv = ex2_approx(s2[c] - m_used[c]);
+                        lsum[c] += pv;
+                    }
+                    *reinterpret_cast<typename E::T*>(pb + c * 128 + ((unit ^ (c & 7)) << 4)) = E::from_float(pv);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[j & 1]);
+            }
+            // l per column: the sum of the 128 threads' partial sums
+            float* rsum = red + 2 * 4 * NQ;
+            if (ok) {
+#pragma unroll
+                for (int c = 0; c < NQ; ++c) {
+                    if (c < G) {
+                        float sm = lsum[c];
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, off);
+                        if (lane == 0) rsum[warp * NQ + c] = sm;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sum_bar);
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(sum_bar, 0, abort_flag));
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(&o_done[(nt - 1) & 1], ((nt - 1) >> 1) & 1, abort_flag));
+            if (ok) {
+                tc_fence_after();
+                uint32_t ov[NQ];
+                tmem_ld_cols<NQ>(o_addr, ov);
+#pragma unroll
+                for (int c = 0; c < NQ; ++c) {
+                    if (c < G) {
+                        const float l = (rsum[c] + rsum[NQ + c]) + (rsum[2 * NQ + c] + rsum[3 * NQ + c]);
+                        p.o_part[((row0 + c) * p.S + split) * D + t] = __uint_as_float(ov[c]) / l;
+                        if (t == c) p.lse_part[(row0 + c) * p.S + split] = (m_used[c] + log2f(l)) * 0.69314718055994530942f;
+                    }
+                }
+            } else {
+                // a wait was abandoned (timeout, recorded in the status word): leave
+                // empty partials (zero weight in the combine) rather than stale memory
+                for (int c = 0; c < G; ++c) p.o_part[((row0 + c) * p.S + split) * D + t] = 0.f;
+                if (t < G) p.lse_part[(row0 + t) * p.S + split] = -INFINITY;
             }
         }
     }

@@ -188,12 +188,15 @@ def test_default_splits(lib):
     f = lib.attn_decode_default_splits
     f.restype = ctypes.c_int
     assert f(0, 32, 8, 100) == 0 and f(1, 30, 8, 100) == 0
-    # B=1, 8 KV heads, 4 query heads each: 8 blocks per split -> one wave of 144
-    assert f(1, 32, 8, 32768) == 18
-    assert f(1, 32, 8, 131072) == 18
-    # B=8: 64 blocks per split; 9 splits = 576 blocks = 3.9 waves of 148
+    # groups of 4 query heads run the keys-as-rows decode, two blocks per SM (296
+    # on B200). B=1, 8 KV heads: 8 blocks per split -> 37 splits = one wave of 296
+    assert f(1, 32, 8, 32768) == 37
+    assert f(1, 32, 8, 131072) == 37
+    # B=8: 64 blocks per split; 9 splits = 576 blocks = 1.95 waves of 296
     assert f(8, 32, 8, 32768) == 9
-    assert f(8, 32, 8, 131072) == 16
+    assert f(8, 32, 8, 131072) == 9
+    # a group of 64 query heads runs the query-rows decode, one block per SM
+    assert f(1, 64, 1, 1000) == 8
     assert f(1, 1, 1, 1) == 1
     for L in (1, 31, 257, 100000):
         s = f(2, 16, 4, L)

@@ -37,8 +37,11 @@ def gpu_combine(o_part, lse_part):
 
 @pytest.mark.parametrize("B,Hq,Hkv,L,d", [(1, 32, 8, 4096, 128), (2, 8, 8, 1000, 128), (2, 4, 1, 777, 64),
                                           (1, 6, 2, 300, 128), (1, 3, 1, 513, 64), (3, 16, 2, 2049, 128),
-                                          (1, 2, 2, 1, 128), (1, 4, 4, 31, 64)])
+                                          (1, 2, 2, 1, 128), (1, 4, 4, 31, 64), (1, 24, 1, 1500, 128),
+                                          (2, 40, 2, 900, 128), (1, 32, 1, 1000, 128), (1, 64, 1, 700, 128)])
 def test_decode_full(B, Hq, Hkv, L, d):
+    """Group sizes G = Hq / Hkv from 1 to 64: up to 32 at d = 128 the kernel with the
+    keys as tile rows (16 or 32 query columns), otherwise the query heads as rows."""
     q, k, v = si.make_decode(5000 + L, B, Hq, Hkv, L, d)
     S = eab.attn_decode_default_splits(B, Hq, Hkv, L)
     chunk = eab.decode_chunk(L, S)
@@ -63,6 +66,23 @@ def test_split_count_sweep(S):
     o, lse = gpu_combine(op, lp)
     o_ref, lse_ref = oracle.decode(q, k, v, d ** -0.5)
     assert_attn_close(o, lse, o_ref, lse_ref, f"S={S}")
+
+
+@pytest.mark.parametrize("G", [4, 24])
+def test_decode_large_logits(G):
+    """Q x 8 (exact in bf16): the running maximum of a query column jumps between
+    key tiles, so the lazy rescale of O runs; partials and the merge against the oracle."""
+    B, Hkv, L, d = 1, 2, 3000, 128
+    q, k, v = si.make_decode(5150 + G, B, G * Hkv, Hkv, L, d)
+    q = (q.float() * 8).to(torch.bfloat16)
+    S = 5
+    chunk = eab.decode_chunk(L, S)
+    op, lp = gpu_partials(q, k, v, S, d ** -0.5)
+    op_ref, lp_ref = oracle.decode_partials(q, k, v, d ** -0.5, S, chunk)
+    assert_attn_close(op.cpu(), lp.cpu(), op_ref, lp_ref, f"partials Qx8 G{G}")
+    o, lse = gpu_combine(op, lp)
+    o_ref, lse_ref = oracle.decode(q, k, v, d ** -0.5)
+    assert_attn_close(o, lse, o_ref, lse_ref, f"decode Qx8 G{G}")
 
 
 def test_combine_alone():
