@@ -16,6 +16,7 @@ place of pointers; ``stream`` defaults to torch's current stream):
     attn_merge(o_acc, lse_acc, o_blk, lse_blk, out=None, init=False)
     attn_bwd(q, k, v, o, lse, dout, delta, dq, dk, dv, causal, scale)   (gradients)
     attn_quant_fp8(x, codes, scales, per_plane=False, transpose=False)  (E4M3 block quantisation)
+    attn_quant_fp8_rotate(x, signs, codes, scales)  (the same after incoherent processing)
     attn_fwd_fp8(q8, k8, vt8, sq, sk, sv, o, lse, causal, scale)        (forward on E4M3 codes)
 Ring attention (context parallelism, ``ring.py``): each rank attends its query
 shard to every key/value shard as the shards travel around the ring of ranks,
@@ -26,7 +27,7 @@ Convenience wrappers that allocate the outputs with torch:
     decode(q, k, v, scale=None, num_splits=None) -> (o, lse)
     attention_backward(q, k, v, o, lse, dout, causal=False, scale=None) -> (dq, dk, dv)
     quantize_fp8(x, per_plane=False, transpose=False) -> (codes, scales)
-    attention_fp8(q, k, v, causal=False, scale=None) -> (o, lse)
+    attention_fp8(q, k, v, causal=False, scale=None, signs=None) -> (o, lse)
 """
 from ._binding import (  # noqa: F401
     AttnError,
@@ -47,11 +48,13 @@ from ._binding import (  # noqa: F401
     attn_fwd_fp8,
     attn_merge,
     attn_quant_fp8,
+    attn_quant_fp8_rotate,
     attn_selftest_bounded_wait,
     attn_status_string,
     decode,
     decode_chunk,
     library_path,
     quantize_fp8,
+    quantize_fp8_rotated,
 )
 from .ring import ring_attention, ring_attention_emulated, ring_schedule  # noqa: F401,E402

@@ -60,6 +60,8 @@ def _load():
     lib.attn_bwd.restype = I
     lib.attn_quant_fp8.argtypes = [P, P, P, I, I, I, I, I, P]
     lib.attn_quant_fp8.restype = I
+    lib.attn_quant_fp8_rotate.argtypes = [P, P, P, P, I, I, I, P]
+    lib.attn_quant_fp8_rotate.restype = I
     lib.attn_fwd_fp8.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.attn_fwd_fp8.restype = I
     return lib
@@ -171,6 +173,25 @@ def attn_quant_fp8(x, codes, scales, per_plane: bool = False, transpose: bool = 
         raise ValueError("attn_quant_fp8: inconsistent shapes")
     _check(_lib.attn_quant_fp8(_ptr(x), _ptr(codes), _ptr(scales), planes, N, d, int(bool(per_plane)),
                                int(bool(transpose)), _stream(stream)), "attn_quant_fp8")
+
+
+def attn_quant_fp8_rotate(x, signs, codes, scales, stream=None):
+    """E4M3 block quantisation (per 128-row block, row-major codes) of x [..., N, d]
+    bf16 after the incoherent-processing rotation y = H (signs o x) / sqrt(d);
+    signs [d] fp32 of +1 / -1."""
+    _need(x, torch.bfloat16, "x")
+    _need(signs, torch.float32, "signs")
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.float32, "scales")
+    *lead, N, d = x.shape
+    planes = 1
+    for n in lead:
+        planes *= n
+    if tuple(signs.shape) != (d,) or tuple(codes.shape) != tuple(x.shape) or \
+            tuple(scales.shape) != (*lead, -(-N // 128)):
+        raise ValueError("attn_quant_fp8_rotate: inconsistent shapes")
+    _check(_lib.attn_quant_fp8_rotate(_ptr(x), _ptr(signs), _ptr(codes), _ptr(scales), planes, N, d,
+                                      _stream(stream)), "attn_quant_fp8_rotate")
 
 
 def attn_fwd_fp8(q8, k8, vt8, sq, sk, sv, o, lse, causal: bool, scale: float, stream=None):
@@ -313,13 +334,28 @@ def quantize_fp8(x, per_plane: bool = False, transpose: bool = False, stream=Non
     return codes, scales
 
 
-def attention_fp8(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
+def quantize_fp8_rotated(x, signs, stream=None):
+    """Allocates and fills (codes, scales) for attn_quant_fp8_rotate."""
+    *lead, N, d = x.shape
+    codes = torch.empty(tuple(x.shape), device=x.device, dtype=torch.uint8)
+    scales = torch.empty(*lead, -(-N // 128), device=x.device, dtype=torch.float32)
+    attn_quant_fp8_rotate(x, signs, codes, scales, stream)
+    return codes, scales
+
+
+def attention_fp8(q, k, v, causal: bool = False, scale: float | None = None, signs=None, stream=None):
     """FP8 forward from bf16 q, k, v: quantises Q and K per 128-row block and V
-    per plane (transposed), then runs attn_fwd_fp8. Returns (o bf16, lse fp32)."""
+    per plane (transposed), then runs attn_fwd_fp8. With ``signs`` ([d] fp32 of
+    +1 / -1, drawn by the caller) Q and K are rotated first (incoherent
+    processing), which leaves Q K^T unchanged. Returns (o bf16, lse fp32)."""
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[-1])
-    q8, sq = quantize_fp8(q, stream=stream)
-    k8, sk = quantize_fp8(k, stream=stream)
+    if signs is None:
+        q8, sq = quantize_fp8(q, stream=stream)
+        k8, sk = quantize_fp8(k, stream=stream)
+    else:
+        q8, sq = quantize_fp8_rotated(q, signs, stream=stream)
+        k8, sk = quantize_fp8_rotated(k, signs, stream=stream)
     vt8, sv = quantize_fp8(v, per_plane=True, transpose=True, stream=stream)
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)

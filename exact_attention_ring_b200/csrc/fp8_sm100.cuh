@@ -1,8 +1,9 @@
 // FP8 (E4M3) forward pass on sm_100a: block quantisation of Q, K, V and the
 // attention forward on the quantised tiles.
 //
-// FlashAttention-3 page: FP8 computation through block quantisation (its
-// other ingredient, incoherent processing, is not built here). Reading taken
+// FlashAttention-3 page: FP8 computation through block quantisation and
+// incoherent processing (a random orthogonal rotation of Q and K that spreads
+// outlier coordinates before they are quantised). Reading taken
 // where the page gives no detail: one fp32 scale per block of 128 consecutive
 // rows of a (batch, head) plane, s = amax / 448 (s = 1 for an all-zero block),
 // code = E4M3(x / s), round to nearest even, divisions in IEEE fp32. Q and K
@@ -12,6 +13,8 @@
 // operand like Q and K.
 //
 // Kernels:
+//   fp8_quant_rows_kernel  per-block scales and row-major codes of Q or K in
+//                        one pass, optionally after the rotation
 //   fp8_amax_kernel      largest |x| per (plane, 128-row block), into scales
 //   fp8_quant_kernel     codes from x and the block (or plane) maximum,
 //                        row-major or transposed
@@ -25,8 +28,12 @@
 //                        O += P8 V8 with both operands K-major in shared
 //                        memory; O x s_v / l and the LSE in the epilogue.
 // The attention kernel: 192 threads, warps 0-3 softmax (thread = query row =
-// TMEM lane), warp 4 the MMA issuer, warp 5 the TMA producer. S is double
-// buffered in TMEM, K/V tiles go through a 3-slot ring, P through two buffers.
+// TMEM lane), warp 4 the MMA issuer, warp 5 the TMA producer. The softmax reads
+// S into registers at once, so one S buffer in TMEM suffices (S(j+1) is
+// computed while the softmax works on tile j); K/V tiles go through a 2-slot
+// ring and P through one shared-memory tile, so that two blocks share an SM (256
+// TMEM columns, about 97 KB of shared memory each): one block's MMAs overlap the
+// other's softmax.
 // O is rescaled lazily: only when a row's running maximum grows by more than
 // 8 (log2 units), so P stays at most 2^8, inside E4M3's range. Every wait is
 // bounded.
@@ -62,7 +69,109 @@ struct QuantParams {
     uint8_t* codes;          // [planes, N, D], or [planes, D, Np] when transposed
     float* scales;           // [planes, nblk]: maxima after the first kernel, scales after the last
     int planes, N, nblk, Np, per_plane;
+    const float* signs;      // [D] +1 / -1: the random signs of the rotation (fp8_quant_rows_kernel<D, true>)
+    float rot_scale;         // fp32 value nearest 1 / sqrt(D)
 };
+
+// One pass over one 128-row block of a plane, for the per-block, row-major codes
+// of Q and K: each warp holds 16 rows in registers (lane l has elements
+// l*E .. l*E+E-1, E = D/32), optionally applies the rotation of incoherent
+// processing (FlashAttention-3 page, FP8 paragraph; reading: y = H (sigma o x) /
+// sqrt(D), H the Sylvester Hadamard matrix, sigma random signs shared by Q and
+// K), then takes the block maximum, its scale and the codes. The rotation is the
+// fast Walsh-Hadamard transform in fp32 with butterflies (a, b) -> (a + b, a - b)
+// of span 1, 2, ..., D/2 in that order (spans below E inside a lane, the rest
+// across lanes by shuffles) and one multiplication by rot_scale: every element
+// takes exactly the fp32 operations of the transform's definition, in its order.
+template <int D, bool ROTATE>
+__global__ void __launch_bounds__(256) fp8_quant_rows_kernel(const QuantParams p) {
+    constexpr int E = D / 32, RPW = 16;
+    const int blk = blockIdx.x, plane = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r0 = blk * 128, rows = min(128, p.N - r0);
+    const __nv_bfloat16* src = p.x + (static_cast<size_t>(plane) * p.N + r0) * D;
+    float v[RPW][E];
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) {
+        const int r = warp * RPW + i;
+        if (r < rows) {
+            if constexpr (E == 4) {
+                const uint2 u = *reinterpret_cast<const uint2*>(src + static_cast<size_t>(r) * D + lane * E);
+                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+                const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+                v[i][0] = a.x; v[i][1] = a.y; v[i][2] = b.x; v[i][3] = b.y;
+            } else {
+                const uint32_t u = *reinterpret_cast<const uint32_t*>(src + static_cast<size_t>(r) * D + lane * E);
+                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+                v[i][0] = a.x; v[i][1] = a.y;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) v[i][e] = 0.f;
+        }
+    }
+    if constexpr (ROTATE) {
+        float sg[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) sg[e] = p.signs[lane * E + e];
+#pragma unroll
+        for (int i = 0; i < RPW; ++i) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) v[i][e] = sg[e] * v[i][e];
+#pragma unroll
+            for (int h = 1; h < E; h *= 2)
+#pragma unroll
+                for (int b = 0; b < E; b += 2 * h)
+#pragma unroll
+                    for (int t = b; t < b + h; ++t) {
+                        const float a = v[i][t], c = v[i][t + h];
+                        v[i][t] = __fadd_rn(a, c);
+                        v[i][t + h] = __fsub_rn(a, c);
+                    }
+#pragma unroll
+            for (int h = E; h < D; h *= 2) {
+                const int m = h / E;  // partner lane of element lane*E + e is lane ^ m
+                const bool lower = (lane & m) == 0;
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const float u = __shfl_xor_sync(0xffffffffu, v[i][e], m);
+                    v[i][e] = lower ? __fadd_rn(v[i][e], u) : __fsub_rn(u, v[i][e]);
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e) v[i][e] = __fmul_rn(v[i][e], p.rot_scale);
+        }
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < RPW; ++i)
+#pragma unroll
+        for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(v[i][e]));  // rows past N hold zeros
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    __shared__ float wm[8];
+    if (lane == 0) wm[warp] = m;
+    __syncthreads();
+    float amax = wm[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) amax = fmaxf(amax, wm[w]);
+    const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    if (threadIdx.x == 0) p.scales[static_cast<size_t>(plane) * p.nblk + blk] = sc;
+    uint8_t* dst = p.codes + (static_cast<size_t>(plane) * p.N + r0) * D;
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) {
+        const int r = warp * RPW + i;
+        if (r >= rows) break;
+        if constexpr (E == 4) {
+            const uint32_t c = uint32_t(e4m3x2(__fdiv_rn(v[i][0], sc), __fdiv_rn(v[i][1], sc))) |
+                               (uint32_t(e4m3x2(__fdiv_rn(v[i][2], sc), __fdiv_rn(v[i][3], sc))) << 16);
+            *reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(r) * D + lane * E) = c;
+        } else {
+            *reinterpret_cast<uint16_t*>(dst + static_cast<size_t>(r) * D + lane * E) =
+                e4m3x2(__fdiv_rn(v[i][0], sc), __fdiv_rn(v[i][1], sc));
+        }
+    }
+}
 
 template <int D>
 __global__ void __launch_bounds__(256) fp8_amax_kernel(const QuantParams p) {
@@ -177,15 +286,17 @@ struct Fp8Params {
 };
 
 struct Fp8Cfg {
-    static constexpr int D = 128, BM = 128, BN = 128, STAGES = 3;
+    static constexpr int D = 128, BM = 128, BN = 128, STAGES = 2;
     static constexpr int TILE = 128 * 128;  // bytes of one 128 x 128 E4M3 tile
     static constexpr int NUM_THREADS = 192;
-    // [Q][K x STAGES][V x STAGES][P x 2][barriers]
-    static constexpr int SMEM_BYTES = 1024 + TILE * (1 + 2 * STAGES + 2) + 32 * 8 + 16;
+    static constexpr uint32_t TMEM_COLS = 256;  // S [0, 128), O [128, 256)
+    // [Q][K x STAGES][V x STAGES][P][barriers]: two blocks fit one SM (shared
+    // memory and TMEM), so one block's MMAs overlap the other's softmax
+    static constexpr int SMEM_BYTES = 1024 + TILE * (1 + 2 * STAGES + 1) + 16 * 8 + 16;
 };
 
 template <bool CAUSAL>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, 2)
     attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_vt, const Fp8Params p) {
     using C = Fp8Cfg;
@@ -195,17 +306,17 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* sQ = smem;
     uint8_t* sK = sQ + TILE;               // [STAGES]
     uint8_t* sV = sK + STAGES * TILE;      // [STAGES], rows = head dimension, 128 keys each
-    uint8_t* sP = sV + STAGES * TILE;      // [2]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * TILE);
+    uint8_t* sP = sV + STAGES * TILE;      // P (E4M3), 128 rows of 128 keys
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sP + TILE);
     uint64_t* q_full = bars;               // Q tile loaded
     uint64_t* kv_full = bars + 1;          // [STAGES] K and V tiles of a slot loaded
-    uint64_t* kv_empty = bars + 4;         // [STAGES] slot read by S and P V
-    uint64_t* s_full = bars + 7;           // [2] S buffer complete
-    uint64_t* s_free = bars + 9;           // [2] S buffer read into registers (4 warp arrivals)
-    uint64_t* p_full = bars + 11;          // [2] P buffer written (4 warp arrivals)
-    uint64_t* pv_done = bars + 13;         // [2] P V of the buffer complete
-    uint64_t* fin = bars + 15;             // every MMA done
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16);
+    uint64_t* kv_empty = bars + 3;         // [STAGES] slot read by S and P V
+    uint64_t* s_full = bars + 5;           // S complete
+    uint64_t* s_free = bars + 6;           // S read into registers (4 warp arrivals)
+    uint64_t* p_full = bars + 7;           // P written (4 warp arrivals)
+    uint64_t* pv_done = bars + 8;          // P V complete
+    uint64_t* fin = bars + 9;              // every MMA done
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 10);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -221,24 +332,22 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&kv_full[i], 1);
             mbar_init(&kv_empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1);
-            mbar_init(&s_free[i], 4);
-            mbar_init(&p_full[i], 4);
-            mbar_init(&pv_done[i], 1);
-        }
+        mbar_init(s_full, 1);
+        mbar_init(s_free, 4);
+        mbar_init(p_full, 4);
+        mbar_init(pv_done, 1);
         mbar_init(fin, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 4) {
-        tmem_alloc(tmem_holder, 512);
+        tmem_alloc(tmem_holder, C::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_holder;  // S buffers at columns 0 and 128, O at 256
+    const uint32_t tmem = *tmem_holder;
 
     if (warp == 5) {
         // ------------------------------------------------------ producer ----
@@ -265,38 +374,38 @@ __global__ void __launch_bounds__(192, 1)
             constexpr uint32_t idesc = make_idesc(128, 128, 0, 0, 0);
             const uint32_t q_addr = smem_addr(sQ);
             auto issue_s = [&](int j) -> bool {
-                const int slot = j % STAGES, sb = j & 1;
+                const int slot = j % STAGES;
                 if (!mbar_wait(&kv_full[slot], (j / STAGES) & 1, abort_flag)) return false;
-                if (j >= 2 && !mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1, abort_flag)) return false;
+                // the softmax has read S(j - 1) into registers
+                if (j >= 1 && !mbar_wait(s_free, (j - 1) & 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t k_addr = smem_addr(sK + slot * TILE);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)  // 32 bytes = 32 elements of K per MMA
-                    mma_f8_ss(tmem + sb * 128, make_sdesc_sw128(q_addr + kk * 32, 16, 1024),
+                    mma_f8_ss(tmem, make_sdesc_sw128(q_addr + kk * 32, 16, 1024),
                               make_sdesc_sw128(k_addr + kk * 32, 16, 1024), idesc, kk > 0 ? 1u : 0u);
-                tc_commit(&s_full[sb]);
+                tc_commit(s_full);
                 return true;
             };
             bool ok = mbar_wait(q_full, 0, abort_flag) && issue_s(0);
             for (int j = 0; ok && j < nk; ++j) {
-                // S(j + 1) goes ahead of P V(j) so that it is ready when the
-                // softmax finishes P(j)
+                // S(j + 1) goes ahead of P V(j): it runs while the softmax works on P(j)
                 if (j + 1 < nk && !issue_s(j + 1)) {
                     ok = false;
                     break;
                 }
-                const int slot = j % STAGES, pb = j & 1;
-                if (!mbar_wait_spin(&p_full[pb], (j >> 1) & 1, abort_flag)) {
+                const int slot = j % STAGES;
+                if (!mbar_wait_spin(p_full, j & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t p_addr = smem_addr(sP + pb * TILE), v_addr = smem_addr(sV + slot * TILE);
+                const uint32_t p_addr = smem_addr(sP), v_addr = smem_addr(sV + slot * TILE);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_f8_ss(tmem + 256, make_sdesc_sw128(p_addr + kk * 32, 16, 1024),
+                    mma_f8_ss(tmem + 128, make_sdesc_sw128(p_addr + kk * 32, 16, 1024),
                               make_sdesc_sw128(v_addr + kk * 32, 16, 1024), idesc, (j > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(&pv_done[pb]);
+                tc_commit(pv_done);
                 tc_commit(&kv_empty[slot]);
             }
             tc_commit(fin);
@@ -313,29 +422,30 @@ __global__ void __launch_bounds__(192, 1)
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nk; ++j) {
-            const int sb = j & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (j >> 1) & 1, abort_flag))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(s_full, j & 1, abort_flag))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            uint32_t sr0[64], sr1[64];
-            tmem_ld64(tmem + lb + sb * 128, sr0);
-            tmem_ld64(tmem + lb + sb * 128 + 64, sr1);
+            uint32_t sr[128];
+            tmem_ld64(tmem + lb, reinterpret_cast<uint32_t(&)[64]>(sr[0]));
+            tmem_ld64(tmem + lb + 64, reinterpret_cast<uint32_t(&)[64]>(sr[64]));
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[sb]);
-            // scores in log2 units: S8 x s_q x s_k(j) x scale x log2(e)
+            if (lane == 0) mbar_arrive(s_free);  // S(j + 1) may overwrite S now
+            // scores in log2 units: S8 x s_q x s_k(j) x scale x log2(e), c > 0
             const float c = p.scale_log2 * sq * skp[j];
             const int k0 = j * 128;
             const int lim = min(p.N - k0, CAUSAL ? q_row - k0 + 1 : 128);  // visible keys: col < lim
-            float x[128];
-            float tmax = -INFINITY;
+            if (__any_sync(0xffffffffu, lim < 128)) {
 #pragma unroll
-            for (int i = 0; i < 128; ++i) {
-                x[i] = i < lim ? __uint_as_float(i < 64 ? sr0[i] : sr1[i - 64]) * c : -INFINITY;
-                tmax = fmaxf(tmax, x[i]);
+                for (int i = 0; i < 128; ++i)
+                    if (i >= lim) sr[i] = 0xff800000u;  // -inf: exp2 gives 0
             }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 128; i += 2) mx = max3(mx, __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
+            const float tmax = mx * c;
             float factor = 1.f;
             if (j == 0) {
                 m_used = tmax;
@@ -343,43 +453,43 @@ __global__ void __launch_bounds__(192, 1)
                 factor = ex2_approx(m_used - tmax);
                 m_used = tmax;
             }
-            float rs = 0.f;
+            const float2 cc2 = make_float2(c, c), negm2 = make_float2(-m_used, -m_used);
+            float2 rsum[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) rsum[k] = make_float2(0.f, 0.f);
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 128; i += 4) {
-                const float p0 = ex2_approx(x[i] - m_used), p1 = ex2_approx(x[i + 1] - m_used);
-                const float p2 = ex2_approx(x[i + 2] - m_used), p3 = ex2_approx(x[i + 3] - m_used);
-                rs += (p0 + p1) + (p2 + p3);
-                pk[i / 4] = uint32_t(e4m3x2(p0, p1)) | (uint32_t(e4m3x2(p2, p3)) << 16);
+                const float2 y0 = ffma2(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), cc2, negm2);
+                const float2 y1 = ffma2(make_float2(__uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3])), cc2, negm2);
+                const float2 p0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
+                const float2 p1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
+                rsum[(i >> 2) & 3] = fadd2(rsum[(i >> 2) & 3], fadd2(p0, p1));
+                pk[i / 4] = uint32_t(e4m3x2(p0.x, p0.y)) | (uint32_t(e4m3x2(p1.x, p1.y)) << 16);
             }
-            l = l * factor + rs;
-            // P buffer sb was last read by P V(j - 2); O must hold every earlier
-            // P V before it is rescaled
-            const bool rescale = __any_sync(0xffffffffu, factor != 1.f);
-            bool w_ok = true;
-            if (rescale && j >= 1)
-                w_ok = mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag);
-            else if (j >= 2)
-                w_ok = mbar_wait(&pv_done[sb], ((j >> 1) - 1) & 1, abort_flag);
-            if (!__all_sync(0xffffffffu, w_ok)) {
+            const float2 rs = fadd2(fadd2(rsum[0], rsum[1]), fadd2(rsum[2], rsum[3]));
+            l = l * factor + (rs.x + rs.y);
+            // P V(j - 1) must be complete: it still reads the P buffer, and O must
+            // hold it before a rescale
+            if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, abort_flag))) {
                 ok = false;
                 break;
             }
-            if (rescale) {
+            if (__any_sync(0xffffffffu, factor != 1.f)) {
                 tc_fence_after();
 #pragma unroll
                 for (int cch = 0; cch < 4; ++cch) {
                     uint32_t ov[32];
-                    tmem_ld32(tmem + lb + 256 + cch * 32, ov);
+                    tmem_ld32(tmem + lb + 128 + cch * 32, ov);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * factor);
-                    tmem_st32(tmem + lb + 256 + cch * 32, ov);
+                    tmem_st32(tmem + lb + 128 + cch * 32, ov);
                 }
                 tmem_st_wait();
             }
             // P row into the 128-byte-swizzled K-major tile: 16-byte chunk cc of
             // row r sits at chunk position cc ^ (r & 7)
-            uint8_t* prow = sP + sb * TILE + r * 128;
+            uint8_t* prow = sP + r * 128;
 #pragma unroll
             for (int cc = 0; cc < 8; ++cc)
                 *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
@@ -387,7 +497,7 @@ __global__ void __launch_bounds__(192, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[sb]);
+            if (lane == 0) mbar_arrive(p_full);
         }
         // epilogue: O x s_v / l in bf16, LSE = ln 2 (m + log2 l)
         if (ok && __all_sync(0xffffffffu, mbar_wait(fin, 0, abort_flag))) {
@@ -397,7 +507,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int cch = 0; cch < 4; ++cch) {
                 uint32_t ov[32];
-                tmem_ld32(tmem + lb + 256 + cch * 32, ov);
+                tmem_ld32(tmem + lb + 128 + cch * 32, ov);
                 if (q_row < p.N) {
 #pragma unroll
                     for (int i = 0; i < 32; i += 8)
@@ -417,7 +527,7 @@ __global__ void __launch_bounds__(192, 1)
     __syncthreads();
     if (warp == 4) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, C::TMEM_COLS);
     }
 }
 

@@ -12,8 +12,9 @@
  * long sequence across devices and merges each device's per-shard results the
  * same way (attn_fwd_f32, attn_merge; FlashAttention-3 page, RingAttention).
  * The backward pass (attn_bwd) recomputes P from the saved log-sum-exp; the
- * FP8 forward (attn_quant_fp8, attn_fwd_fp8) runs on block-quantised E4M3
- * inputs (FlashAttention-3 page).
+ * FP8 forward (attn_quant_fp8, attn_quant_fp8_rotate, attn_fwd_fp8) runs on
+ * block-quantised E4M3 inputs, optionally after incoherent processing
+ * (FlashAttention-3 page).
  *
  * Conventions shared by every call:
  *  - All tensors are dense, contiguous, row-major device buffers owned by the
@@ -95,6 +96,9 @@ attn_status_t attn_fwd_f32(const void* q, const void* k, const void* v, float* o
  *  S = num_splits, 1 <= S <= L. Split s covers keys [s*C, min(L, (s+1)*C)) with
  *  C = 128 * ceil(ceil(L / S) / 128). A split with no keys gets lse = -inf, o = 0.
  *  d 64 or 128; Hq % Hkv == 0; scale finite and > 0.
+ *  If a bounded wait inside the kernel runs out (attn_device_status then reports
+ *  ATTN_ERR_TIMEOUT), the splits it abandoned are written as empty (lse = -inf,
+ *  o = 0): the results of that call are not attention and must be discarded.
  */
 attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v,
                                   float* o_part, float* lse_part,
@@ -112,7 +116,9 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v,
  *  lse_part [B, Hq, S]    fp32 (device, read)
  *  o        [B, Hq, d]    bf16 (device, written)
  *  lse      [B, Hq]       fp32 (device, written)
- *  d 64 or 128; S >= 1; at least one split of every (b, h) must be non-empty.
+ *  d 64 or 128; 1 <= S <= 12000 (one weight per split is kept in shared
+ *  memory; larger S returns ATTN_ERR_INVALID_ARG); at least one split of
+ *  every (b, h) must be non-empty.
  */
 attn_status_t attn_combine(const float* o_part, const float* lse_part, void* o, float* lse,
                            int B, int Hq, int num_splits, int d, attn_stream_t stream);
@@ -174,9 +180,9 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
                        attn_stream_t stream);
 
 /*
- * attn_quant_fp8, attn_fwd_fp8 — the forward pass on FP8 (E4M3) inputs.
- * FlashAttention-3 page: FP8 computation with block quantisation (incoherent
- * processing, its other ingredient, is not provided). Reading of "block
+ * attn_quant_fp8, attn_quant_fp8_rotate, attn_fwd_fp8 — the forward pass on
+ * FP8 (E4M3) inputs. FlashAttention-3 page: FP8 computation with block
+ * quantisation and incoherent processing. Reading of "block
  * quantisation": one fp32 scale per block of 128 consecutive rows of a
  * (batch, head) plane — or one per plane — s = amax / 448 with amax the
  * largest |x| of the block (s = 1 for an all-zero block), code = E4M3(x / s),
@@ -188,7 +194,25 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
  *          uint8 with Np = 128 * ceil(N / 128), codes of keys >= N zero
  *  scales  [planes, ceil(N / 128)] fp32 (written); with per_plane != 0 every
  *          block of a plane gets the plane's scale
- *  d 64 or 128 (else ATTN_ERR_UNSUPPORTED); planes <= 65535. Three launches.
+ *  d 64 or 128 (else ATTN_ERR_UNSUPPORTED); planes <= 65535. One launch for
+ *  per-block row-major codes (per_plane 0, transpose 0), three otherwise.
+ *
+ * attn_quant_fp8_rotate quantises like attn_quant_fp8 (per_plane 0,
+ * transpose 0) after incoherent processing of every row. Reading of the page's
+ * "incoherent processing" (it gives no detail): each row x of Q and of K is
+ * replaced by y = H (signs o x) / sqrt(d), H the d x d Sylvester Hadamard
+ * matrix and signs a vector of random +1 / -1 shared by Q and K. H H^T = d I,
+ * so the rotation is orthogonal and Q K^T is unchanged, while an outlier in one
+ * coordinate is spread over all d before quantisation. y is computed in fp32
+ * as the fast Walsh-Hadamard transform (butterflies (a, b) -> (a + b, a - b) of
+ * span 1, 2, ..., d/2 in that order) and one multiplication by the fp32 value
+ * nearest 1 / sqrt(d); the codes and scales are those of the block quantisation
+ * of y. Rotate Q and K with the same signs and leave V as it is: attn_fwd_fp8 on
+ * the results computes the attention of the original inputs.
+ *  x       [planes, N, d] bf16 (device, read)
+ *  signs   [d] fp32, each +1 or -1 (device, read; the caller draws them)
+ *  codes   [planes, N, d] uint8 (written), scales [planes, ceil(N / 128)] (written)
+ *  d 64 or 128 (else ATTN_ERR_UNSUPPORTED); planes <= 65535. One launch.
  *
  * attn_fwd_fp8 computes O and LSE (as attn_fwd) from quantised inputs:
  *  q8  [B, Hq, N, 128]  codes from attn_quant_fp8(q, ..., per_plane 0, transpose 0)
@@ -204,6 +228,8 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
  */
 attn_status_t attn_quant_fp8(const void* x, void* codes, float* scales, int planes, int N, int d,
                              int per_plane, int transpose, attn_stream_t stream);
+attn_status_t attn_quant_fp8_rotate(const void* x, const float* signs, void* codes, float* scales,
+                                    int planes, int N, int d, attn_stream_t stream);
 attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* sq,
                            const float* sk, const float* sv, void* o, float* lse,
                            int B, int Hq, int Hkv, int N, int d, int causal, float scale,
@@ -269,15 +295,22 @@ attn_status_t attn_selftest_bounded_wait(int limit_us, attn_stream_t stream);
  *  q [B, Hq, d], k/v [B, Hkv, L, d] bf16 (device, read)
  *  o [B, Hq, d] bf16, lse [B, Hq] fp32 (device, written)
  *  num_splits, d, scale: as for attn_decode_splitkv.
- * Limit: B * Hq * num_splits * (d + 1) <= 1,048,576; larger problems return
- * ATTN_ERR_INVALID_ARG before anything is enqueued (use fewer splits, or the
- * attn_decode_splitkv + attn_combine pair with caller-owned partials).
- * The first call on a device looks up the array's device address once (with
- * that device current); make that first call before any stream capture.
+ * Limit: B * Hq * num_splits * (d + 1) <= 1,048,576 and num_splits <= 12000
+ * (the combine's bound); larger problems, and any argument attn_decode_splitkv
+ * or attn_combine would reject, return ATTN_ERR_INVALID_ARG before anything is
+ * enqueued (use fewer splits, or the attn_decode_splitkv + attn_combine pair
+ * with caller-owned partials).
+ * The first call on a device looks up the array's device address (with that
+ * device current) and the library keeps it for the life of the process; make
+ * that first call before any stream capture. After cudaDeviceReset (or anything
+ * else that tears down and recreates the device's primary context) the kept
+ * address is stale: such a process must not call attn_decode_noalloc again.
  * The call never calls cudaMalloc, cudaFree or any allocating routine. All calls
  * on a device share the one array and it keeps the last call's contents;
  * nothing in it needs clearing, because every partial is written before it is
- * read. Calls that can overlap on the GPU (different streams without ordering
+ * read (a split abandoned after a bounded wait ran out is written as empty, and
+ * attn_device_status reports ATTN_ERR_TIMEOUT: discard that call's o and lse).
+ * Calls that can overlap on the GPU (different streams without ordering
  * between them) race on the array and must not be issued.
  */
 attn_status_t attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -64,6 +64,23 @@ def make_decode(seed: int, B: int, Hq: int, Hkv: int, L: int, d: int, pin: bool 
     return q, k, v
 
 
+def make_signs(seed: int, d: int) -> torch.Tensor:
+    """Random signs (+1 / -1, fp32 [d]) for the incoherent-processing rotation:
+    the method draws them once and shares them between Q and K."""
+    gen = torch.Generator().manual_seed(seed)
+    return torch.where(torch.rand(d, generator=gen) < 0.5, -1.0, 1.0).to(torch.float32)
+
+
+def with_outlier_channels(x: torch.Tensor, channels=((3, 20.0), (77, 15.0))) -> torch.Tensor:
+    """x with a few head-dimension channels scaled up (the outlier features the
+    FP8 rotation is meant for), rounded back to x's type."""
+    xf = x.float().clone()
+    for c, m in channels:
+        if c < xf.shape[-1]:
+            xf[..., c] *= m
+    return xf.to(x.dtype).contiguous()
+
+
 def sample_rows(seed: int, B: int, H: int, N: int, tile: int = 128, per_slice: int = 256,
                 max_slices: int = 4):
     """Flat row indices ((b*H + h)*N + i) for sampled parity checks.

@@ -73,6 +73,29 @@ def test_backward_large_logits(causal):
     _run(1, 4, 4, 512, 128, causal, 3500, q_mult=8.0)
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_backward_bench_shape_sampled_heads(causal):
+    """The bench's backward workload (B2 H32 N2048 d128, every head in one launch
+    set: 64 (batch, head) planes, several waves of the dK/dV and dQ grids),
+    checked on three (batch, head) planes, each against the oracle's backward on
+    that plane alone (with Hq = Hkv the gradients of a plane depend only on it)."""
+    B, H, N, d = 2, 32, 2048, 128
+    q, k, v = si.make_qkv(1001, B, H, H, N, d)
+    do = si.make_dout(1002, B, H, N, d)
+    qg, kg, vg, dog = (t.to(DEV) for t in (q, k, v, do))
+    o, lse = eab.attention(qg, kg, vg, causal=causal)
+    dq, dk, dv = eab.attention_backward(qg, kg, vg, o, lse, dog, causal=causal)
+    torch.cuda.synchronize()
+    assert eab.attn_device_status() == 0
+    for b, h in [(0, 0), (1, 31), (0, 17)]:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        rq, rk, rv = oracle.attention_backward(q[sl], k[sl], v[sl], do[sl], causal, d ** -0.5)
+        tag = f"bench shape causal={causal} plane ({b},{h})"
+        _close(dq[sl], rq, "dq " + tag)
+        _close(dk[sl], rk, "dk " + tag)
+        _close(dv[sl], rv, "dv " + tag)
+
+
 def test_backward_causal_first_row_has_no_dq():
     """Row 0 sees only key 0, so P_00 = 1 and dS_00 = dP_00 - Delta_0 = 0 up to
     rounding: dq of row 0 vanishes next to the other rows'."""
