@@ -12,7 +12,9 @@
 // B200 mapping. A persistent grid (one CTA per SM) walks a list of work items;
 // an item is one 256-row query block of one (batch, head), processed as two
 // 128-row query tiles that share every K/V tile. Causal items are ordered
-// heaviest first and dealt to the CTAs in snake order. 384 threads,
+// heaviest first; non-causal items head by head, so that the query blocks of one
+// head run in the same wave and share its K/V tiles through L2; the list is
+// dealt to the CTAs in snake order. 384 threads,
 // warp-specialised:
 //   warps 0-3   softmax of query tile 0, one thread per row (TMEM lane), and
 //               its epilogue: O/l rounded to the input type (or kept in fp32
@@ -92,10 +94,18 @@ struct FwdItem {
 template <bool CAUSAL>
 __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int w) {
     FwdItem it;
-    const int bh_count = p.B * p.Hq;
-    const int rank = w / bh_count;
-    it.bh = w % bh_count;
-    it.qb = CAUSAL ? (p.n_qblocks - 1 - rank) : rank;  // heaviest causal blocks first
+    if (CAUSAL) {
+        // heaviest blocks first: every (batch, head) at the last query block, then
+        // at the one before, ...
+        const int bh_count = p.B * p.Hq;
+        it.bh = w % bh_count;
+        it.qb = p.n_qblocks - 1 - w / bh_count;
+    } else {
+        // head by head: the query blocks of one head run in the same wave and
+        // read its K/V tiles from L2
+        it.bh = w / p.n_qblocks;
+        it.qb = w % p.n_qblocks;
+    }
     it.b = it.bh / p.Hq;
     it.h = it.bh % p.Hq;
     it.hk = it.h / (p.Hq / p.Hkv);

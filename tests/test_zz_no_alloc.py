@@ -7,8 +7,9 @@ no-allocation entry point keeps the partials in a fixed array compiled into
 the library. This test calls it through the C ABI (ctypes on the shared
 library itself), twice in a row with different problems, and checks each
 result against the existing attn_decode_splitkv + attn_combine pair on the
-same inputs, within the tolerances the other parity tests use. It also checks
-that a problem larger than the fixed array is rejected before any launch.
+same inputs and against the float64 oracle, within the tolerances the other
+parity tests use. It also checks that a problem larger than the fixed array,
+or with more splits than the combine takes, is rejected before any launch.
 
 The file is named so that pytest collects it last.
 """
@@ -17,6 +18,7 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 import seeded_inputs as si
 from attn_check import assert_attn_close
 
@@ -64,6 +66,8 @@ def test_noalloc_matches_existing_entry_point_twice(lib):
         torch.cuda.synchronize()
         assert eab.attn_device_status() == ATTN_OK
         assert_attn_close(o, lse, o_ref.double().cpu(), lse_ref.double().cpu(), f"noalloc B{B} L{L} d{d}")
+        o_or, lse_or = oracle.decode(q.cpu(), k.cpu(), v.cpu(), scale)
+        assert_attn_close(o, lse, o_or, lse_or, f"noalloc vs oracle B{B} L{L} d{d}")
 
 
 def test_noalloc_rejects_problems_beyond_the_array(lib):
@@ -75,3 +79,18 @@ def test_noalloc_rejects_problems_beyond_the_array(lib):
     st, _, _ = _noalloc(lib, q, k, v, S - 1, d ** -0.5)
     assert st == ATTN_OK
     torch.cuda.synchronize()
+
+
+def test_noalloc_rejects_more_splits_than_the_combine_takes(lib):
+    # 12001 splits of a 64-wide head fit the array (12001 * 65 floats) but not the
+    # combine's 12000 per-split weights: rejected before the decode is enqueued
+    B, Hq, Hkv, L, d = 1, 1, 1, 13000, 64
+    q, k, v = (t.cuda() for t in si.make_decode(9300, B, Hq, Hkv, L, d))
+    st, _, _ = _noalloc(lib, q, k, v, 12001, d ** -0.5)
+    assert st == ATTN_ERR_INVALID_ARG
+    st, o, lse = _noalloc(lib, q, k, v, 12000, d ** -0.5)
+    assert st == ATTN_OK
+    torch.cuda.synchronize()
+    assert eab.attn_device_status() == ATTN_OK
+    o_or, lse_or = oracle.decode(q.cpu(), k.cpu(), v.cpu(), d ** -0.5)
+    assert_attn_close(o, lse, o_or, lse_or, "noalloc 12000 splits")
