@@ -7,6 +7,8 @@ One step is one pass of the whole path over one batch of synthetic inputs:
   2. attn_fwd, non-causal, same shape
   3. attn_decode_splitkv + 4. attn_combine on single-query decode
      (B=1, Hq=32, Hkv=8, L=131072, d=128; the default split count).
+After the timed loop the same decode pair at L=32768 for B=1 and B=8 is timed
+alone (L2 flushed before every launch) and reported beside the step's kernels.
 The printed `value` is the causal prefill's TFLOPS (4*B*H*N^2*d/2 per launch
 over the kernel's CUDA-event time, summed over all ranks); the decode's KV-read
 GB/s is reported beside it. Inputs are seeded N(0,1) bf16, resident in HBM
@@ -51,18 +53,26 @@ METRIC = "attn fwd TFLOPS (% BF16 TC peak); split-KV decode GB/s (% HBM peak)"
 PREFILL = si.PrefillShape("llama7b B2 H32 N2048 d128", 2, 32, 32, 2048, 128, True, seed=1001)
 PREFILL_NC = si.PrefillShape("llama7b B2 H32 N2048 d128 non-causal", 2, 32, 32, 2048, 128, False, seed=1001)
 DECODE = si.DecodeShape("decode B1 Hq32 Hkv8 L131072 d128", 1, 32, 8, 131072, 128, seed=1004)
+# every decode the bench times: (kernels key, shape); the first is the step's decode,
+# the others are timed after the step loop
+DECODES = [("decode", DECODE),
+           ("decode_b1_l32k", si.DecodeShape("decode B1 Hq32 Hkv8 L32768 d128", 1, 32, 8, 32768, 128, seed=1005)),
+           ("decode_b8_l32k", si.DecodeShape("decode B8 Hq32 Hkv8 L32768 d128", 8, 32, 8, 32768, 128, seed=1006))]
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch from one ncu capture, valid only for the kernel source
 # it was taken on (sha256 of the kernel file, first 16 hex digits).
 NCU_TRAFFIC = {
-    # decode_splitkv_kernel<128>, B1 Hq32 Hkv8 L131072 d128 (the bench's decode workload)
-    "decode": {"bytes_per_launch": 536948992 + 3485696, "source_sha": "4b6ee8ffded319ea"},
-    # attn_fwd_kernel<128,causal / non-causal>, B2 H32 N2048 d128 (the bench's prefill workloads),
-    # read + write with cold caches (ncu flushes them before each captured launch)
-    "attn_fwd_causal": {"bytes_per_launch": 149111296 + 16082944, "source_sha": "30dee28611453093"},
-    "attn_fwd_noncausal": {"bytes_per_launch": 269126144 + 28518144, "source_sha": "30dee28611453093"},
+    # decode_splitkv_keys_kernel<16,3>: B1 Hq32 Hkv8 L131072 d128 (the step's decode) and the two
+    # L32768 decodes; attn_fwd_kernel<128, causal / non-causal>: B2 H32 N2048 d128. Read + write
+    # with cold caches (ncu flushes them before each captured launch); the prefill's O (33.5 MB)
+    # mostly stays dirty in L2 when the kernel ends, so its write-back is not counted here.
+    "decode": {"bytes_per_launch": 536989440 + 3163904, "source_sha": "e8f2cefbecba28e0"},
+    "decode_b1_l32k": {"bytes_per_launch": 134306560 + 3091456, "source_sha": "e8f2cefbecba28e0"},
+    "decode_b8_l32k": {"bytes_per_launch": 1074017280 + 3969536, "source_sha": "e8f2cefbecba28e0"},
+    "attn_fwd_causal": {"bytes_per_launch": 144750080 + 15959552, "source_sha": "410f38f5c06bc391"},
+    "attn_fwd_noncausal": {"bytes_per_launch": 100970496 + 10457344, "source_sha": "410f38f5c06bc391"},
 }
 
 
@@ -181,7 +191,7 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # ----------------------------------------------------------------- our arm --
 
-def measure_extra_paths(eab, q, k, v, o, lse, p, flush, stream, iters=10, warm=3):
+def measure_extra_paths(eab, q, k, v, o, lse, p, flush_l2, stream, iters=10, warm=3):
     """The backward pass and the FP8 forward on the prefill workload (causal),
     each timed alone with CUDA events after the timed step (L2 flushed before
     every launch); median of `iters` launches."""
@@ -190,7 +200,7 @@ def measure_extra_paths(eab, q, k, v, o, lse, p, flush, stream, iters=10, warm=3
             fn()
         ts = []
         for _ in range(iters):
-            flush.fill_(0.0)
+            flush_l2()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             fn()
@@ -233,15 +243,36 @@ def run_ours(args):
     o2 = torch.empty_like(q)
     lse2 = torch.empty_like(lse)
     dc = DECODE
-    qd, kd, vd = (t.to(dev) for t in si.make_decode(dc.seed + 17 * rank, dc.B, dc.Hq, dc.Hkv, dc.L, dc.d))
-    S = eab.attn_decode_default_splits(dc.B, dc.Hq, dc.Hkv, dc.L)
-    o_part = torch.empty(dc.B, dc.Hq, S, dc.d, device=dev)
-    lse_part = torch.empty(dc.B, dc.Hq, S, device=dev)
-    od = torch.empty(dc.B, dc.Hq, dc.d, device=dev, dtype=torch.bfloat16)
-    lsed = torch.empty(dc.B, dc.Hq, device=dev)
+    dec_sets = []
+    for name, shp in DECODES:
+        qd, kd, vd = (t.to(dev) for t in si.make_decode(shp.seed + 17 * rank, shp.B, shp.Hq, shp.Hkv, shp.L, shp.d))
+        Sd = eab.attn_decode_default_splits(shp.B, shp.Hq, shp.Hkv, shp.L)
+        dec_sets.append(dict(name=name, shape=shp, q=qd, k=kd, v=vd, S=Sd,
+                             o_part=torch.empty(shp.B, shp.Hq, Sd, shp.d, device=dev),
+                             lse_part=torch.empty(shp.B, shp.Hq, Sd, device=dev),
+                             o=torch.empty(shp.B, shp.Hq, shp.d, device=dev, dtype=torch.bfloat16),
+                             lse=torch.empty(shp.B, shp.Hq, device=dev)))
+    S = dec_sets[0]["S"]
     flush = torch.empty(L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
+    flush_read = torch.ones(2 * L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32)  # 512 MB
+    flush_sum = torch.empty((), device=dev, dtype=torch.float32)
 
     n_ev = 5
+    def flush_l2():
+        # write a buffer larger than L2, then read another: the next kernel starts
+        # with none of its inputs in L2 and no dirty lines to write back
+        flush.fill_(float(rank))
+        torch.sum(flush_read, dim=0, out=flush_sum)
+
+    def run_decode(ds, ev=None, i0=0):
+        eab.attn_decode_splitkv(ds["q"], ds["k"], ds["v"], ds["o_part"], ds["lse_part"], ds["S"],
+                                ds["shape"].scale, stream)
+        if ev is not None:
+            ev[i0].record(stream)
+        eab.attn_combine(ds["o_part"], ds["lse_part"], ds["o"], ds["lse"], stream)
+        if ev is not None:
+            ev[i0 + 1].record(stream)
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
@@ -251,13 +282,8 @@ def run_ours(args):
         eab.attn_fwd(q, k, v, o2, lse2, False, p.scale, stream)
         if ev is not None:
             ev[2].record(stream)
-        eab.attn_decode_splitkv(qd, kd, vd, o_part, lse_part, S, dc.scale, stream)
-        if ev is not None:
-            ev[3].record(stream)
-        eab.attn_combine(o_part, lse_part, od, lsed, stream)
-        if ev is not None:
-            ev[4].record(stream)
-        flush.fill_(float(rank))  # write > L2 so the next prefill starts cold
+        run_decode(dec_sets[0], ev, 3)
+        flush_l2()
 
     for _ in range(args.warmup):
         step()
@@ -278,9 +304,24 @@ def run_ours(args):
     total_ms = max_over_ranks(start.elapsed_time(end), world)
     t_fwd_c = sum(e[0].elapsed_time(e[1]) for e in events) / args.steps
     t_fwd_n = sum(e[1].elapsed_time(e[2]) for e in events) / args.steps
-    t_dec = sum(e[2].elapsed_time(e[3]) for e in events) / args.steps
-    t_comb = sum(e[3].elapsed_time(e[4]) for e in events) / args.steps
-    t_fwd_c, t_fwd_n, t_dec, t_comb = (max_over_ranks(x, world) for x in (t_fwd_c, t_fwd_n, t_dec, t_comb))
+    t_fwd_c, t_fwd_n = (max_over_ranks(x, world) for x in (t_fwd_c, t_fwd_n))
+    dec_sets[0]["t_dec"] = max_over_ranks(sum(e[2].elapsed_time(e[3]) for e in events) / args.steps, world)
+    dec_sets[0]["t_comb"] = max_over_ranks(sum(e[3].elapsed_time(e[4]) for e in events) / args.steps, world)
+    t_dec, t_comb = dec_sets[0]["t_dec"], dec_sets[0]["t_comb"]
+    # the L = 32768 decodes, timed alone after the loop: median of 10 launches, each
+    # after a flush (every rank runs the same launches)
+    for ds in dec_sets[1:]:
+        for _ in range(3):
+            run_decode(ds)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(10)]
+        for ev3 in evs:
+            flush_l2()
+            ev3[0].record(stream)
+            run_decode(ds, ev3, 1)
+        torch.cuda.synchronize()
+        ds["t_dec"] = max_over_ranks(statistics.median(e[0].elapsed_time(e[1]) for e in evs), world)
+        ds["t_comb"] = max_over_ranks(statistics.median(e[1].elapsed_time(e[2]) for e in evs), world)
+    assert eab.attn_device_status() == 0
     assert eab.attn_device_status() == 0
 
     tflops_c = p.flops() / (t_fwd_c * 1e-3) / 1e12
@@ -357,10 +398,21 @@ def run_ours(args):
     roof_fwd_nc = {"kernel": "attn_fwd_kernel<128,noncausal>", "bound": "tensor", "achieved": round(tflops_n, 1),
                    "peak": tc_peak, "unit": "TFLOP/s", "frac": round(tflops_n / tc_peak, 4),
                    "traffic": traffic("attn_fwd_noncausal", fwd_sha), "ms": round(t_fwd_n, 5)}
-    roof_dec = {"kernel": "decode_splitkv_kernel<128>", "bound": "hbm", "achieved": round(dec_kernel_gbs, 1),
-                "peak": hbm_peak, "unit": "GB/s", "frac": round(dec_kernel_gbs / hbm_peak, 4),
-                "traffic": traffic("decode", dec_sha), "ms": round(t_dec, 5),
-                "peak_source": f"{peak_src} hbm_gbs"}
+    dec_roofs = {}
+    for ds in dec_sets:
+        shp = ds["shape"]
+        gbs = shp.kv_bytes() / (ds["t_dec"] * 1e-3) / 1e9
+        dec_roofs[ds["name"]] = {
+            "kernel": "decode_splitkv_keys_kernel<16,3> (keys as tile rows)", "bound": "hbm", "achieved": round(gbs, 1),
+            "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4),
+            "traffic": traffic(ds["name"], dec_sha), "ms": round(ds["t_dec"], 5), "ms_combine": round(ds["t_comb"], 5),
+            "with_combine_gbs": round(shp.kv_bytes() / ((ds["t_dec"] + ds["t_comb"]) * 1e-3) / 1e9, 1),
+            "workload": f"B{shp.B} Hq{shp.Hq} Hkv{shp.Hkv} L{shp.L} d{shp.d}, {ds['S']} splits",
+            "peak_source": f"{peak_src} hbm_gbs"}
+    roof_dec = dec_roofs["decode"]
+    for ds in dec_sets[1:]:
+        dec_roofs[ds["name"]]["timed"] = "alone after the step loop, L2 flushed before each launch, median of 10"
+    # the dominant kernel: the one that takes the most time in the step
     times = {"fwd_causal": t_fwd_c, "fwd_noncausal": t_fwd_n, "decode": t_dec}
     dominant = max(times, key=times.get)
     roofline = {"fwd_causal": roof_fwd, "fwd_noncausal": roof_fwd_nc, "decode": roof_dec}[dominant]
@@ -370,7 +422,7 @@ def run_ours(args):
     extra = None
     if world == 1:
         try:
-            t_bwd, t_fp8, t_quant = measure_extra_paths(eab, q, k, v, o, lse, p, flush, stream)
+            t_bwd, t_fp8, t_quant = measure_extra_paths(eab, q, k, v, o, lse, p, flush_l2, stream)
             fl_bwd = 2.5 * p.flops()  # the five N x N x d products of the backward pass
             extra = {
                 "note": "timed alone after the step, same prefill workload (causal), L2 flushed, median of 10",
@@ -404,12 +456,14 @@ def run_ours(args):
             "data": "synthetic (seeded N(0,1), bf16)",
             "config": {
                 "workload": "prefill B2 H32 N2048 d128 causal (LLaMA-7B shape); step also runs the non-causal "
-                            "prefill and split-KV decode B1 Hq32 Hkv8 L131072 d128 + combine",
+                            "prefill and split-KV decode + combine at B1 Hq32 Hkv8 L131072 d128; B1 and B8 "
+                            "L32768 decodes are timed alone after the step loop",
                 "prefill": {"B": p.B, "Hq": p.Hq, "Hkv": p.Hkv, "N": p.N, "d": p.d, "causal": True},
                 "decode": {"B": dc.B, "Hq": dc.Hq, "Hkv": dc.Hkv, "L": dc.L, "d": dc.d, "num_splits": S},
                 "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                "l2": "inputs resident in HBM; a 256 MB buffer write and the 537 MB decode KV stream (> 126 MB L2) "
-                      "run between consecutive prefill launches",
+                "l2": "flushed: between steps a 256 MB buffer write and then a 512 MB buffer read (> 126 MB L2), "
+                      "so each prefill starts with a cold L2 holding no dirty lines; the step's decode K/V (537 MB) "
+                      "is cold; the L32768 decodes get the same flush before each launch",
             },
             "decode": {"value": round(dec_gbs * world, 1), "unit": "GB/s", "kernel_gbs": round(dec_kernel_gbs, 1),
                        "frac_hbm": round(dec_kernel_gbs / hbm_peak, 4), "ms_decode": round(t_dec, 5),
@@ -417,7 +471,7 @@ def run_ours(args):
             "prefill_noncausal": {"value": round(tflops_n * world, 2), "unit": "TFLOPS",
                                   "frac": round(tflops_n / tc_peak, 4)},
             "roofline": roofline,
-            "kernels": {"fwd_causal": roof_fwd, "fwd_noncausal": roof_fwd_nc, "decode": roof_dec},
+            "kernels": {"fwd_causal": roof_fwd, "fwd_noncausal": roof_fwd_nc, **dec_roofs},
             "e2e": {"value": round(p.flops() * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
                     "pipeline": "per step: H2D of q,k,v, attn_fwd, D2H of o,lse; copies on their own streams, "
