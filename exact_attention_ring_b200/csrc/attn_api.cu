@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -158,6 +159,10 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
     if (items > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
     p.n_items = static_cast<int>(items);
     p.scale_log2 = scale * kLog2e;
+    // each non-causal launch counts its work items in its own slot; launches that
+    // use one slot at the same time (kFwdSchedSlots launches in flight) would share it
+    static std::atomic<unsigned int> launch_seq{0};
+    p.sched_slot = static_cast<int>(launch_seq.fetch_add(1u) % kFwdSchedSlots);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d == 128)
         return causal ? launch_fwd<128, true, F32OUT, E>(tq, tk, tv, p, st)

@@ -12,9 +12,12 @@
 // B200 mapping. A persistent grid (one CTA per SM) walks a list of work items;
 // an item is one 256-row query block of one (batch, head), processed as two
 // 128-row query tiles that share every K/V tile. Causal items are ordered
-// heaviest first; non-causal items head by head, so that the query blocks of one
-// head run in the same wave and share its K/V tiles through L2; the list is
-// dealt to the CTAs in snake order. 384 threads,
+// heaviest first and dealt to the CTAs in snake order; non-causal items head by
+// head, so that the query blocks of one head run in the same wave and share its
+// K/V tiles through L2, and a CTA takes its first item by its index and each
+// later one from a per-launch counter (the first producer thread takes it and
+// hands it to the other roles through a small ring in shared memory), so the
+// CTAs finish together. 384 threads,
 // warp-specialised:
 //   warps 0-3   softmax of query tile 0, one thread per row (TMEM lane), and
 //               its epilogue: O/l rounded to the input type (or kept in fp32
@@ -63,7 +66,19 @@ struct FwdParams {
     int n_qblocks;     // ceil(N / 256)
     int n_items;       // n_qblocks * B * Hq
     float scale_log2;  // scale * log2(e)
+    int sched_slot;    // this launch's work counter in g_fwd_sched
 };
+
+// Dynamic work distribution (non-causal launches): a CTA takes its first item by
+// its index and every later one from a counter, in the list's order, so the
+// CTAs finish together whatever each item actually costs. Each launch uses its
+// own counter slot (the host cycles through them); the last CTA to finish resets
+// the slot to zero for its next use. Causal launches deal their items statically
+// (fwd_work_index): with items from 31 down to 3 key-tile units, heaviest first,
+// the static snake order already reaches the makespan of a greedy longest-first
+// schedule and saves the counter's hand-over at every item.
+constexpr int kFwdSchedSlots = 64;
+__device__ unsigned int g_fwd_sched[kFwdSchedSlots][2];  // [items taken past the first round, CTAs done]
 
 template <int D>
 struct FwdCfg {
@@ -77,13 +92,25 @@ struct FwdCfg {
     static constexpr int STAGE_O_BYTES = 32 * 64 * 2;  // per softmax warp: 32 rows x 64 bf16
     static constexpr int NUM_THREADS = 384;
     static constexpr int NUM_PRODUCERS = 2;
-    // q_full, q_empty, slot_full, slot_empty, s_full, p_full, o_done, o_free, turn, drain, p_half
-    static constexpr int NUM_BARRIERS = 2 * 2 + 2 * SLOTS + 7 * 2;
-    static constexpr int SMEM_BYTES =
-        1024 + TILES * Q_TILE_BYTES + SLOTS * TILE_BYTES + 8 * STAGE_O_BYTES + NUM_BARRIERS * 8 + 16;
+    static constexpr int ITEM_RING = 4;  // work items handed from the fetching thread to the other roles
+    // q_full, q_empty, slot_full, slot_empty, s_full, p_full, o_done, o_free, turn, drain, p_half,
+    // item_full, item_empty
+    static constexpr int NUM_BARRIERS = 2 * 2 + 2 * SLOTS + 7 * 2 + 2 * ITEM_RING;
+    // item readers: the second producer, the two MMA issuers and the eight softmax warps
+    static constexpr int ITEM_READERS = 11;
+    static constexpr int SMEM_BYTES = 1024 + TILES * Q_TILE_BYTES + SLOTS * TILE_BYTES + 8 * STAGE_O_BYTES +
+                                      NUM_BARRIERS * 8 + 16 + ITEM_RING * 4;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: P <= 2^8 between rescales
 };
+
+// The r-th item of this CTA in the static deal: rounds of gridDim.x items, dealt
+// forwards in even rounds and backwards in odd ones. Past the last item of this
+// CTA every later round is past the end too.
+__device__ __forceinline__ int fwd_work_index(int r) {
+    const int G = gridDim.x, c = blockIdx.x;
+    return r * G + ((r & 1) ? (G - 1 - c) : c);
+}
 
 // One work item: a 256-row query block of one (batch, head).
 struct FwdItem {
@@ -115,13 +142,6 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int w) {
     return it;
 }
 
-// The r-th work item of this CTA: rounds of gridDim.x items, dealt forwards in
-// even rounds and backwards in odd ones. Past the last item of this CTA every
-// later round is past the end too.
-__device__ __forceinline__ int fwd_work_index(int r) {
-    const int G = gridDim.x, c = blockIdx.x;
-    return r * G + ((r & 1) ? (G - 1 - c) : c);
-}
 
 // Max of 64 values with eight independent chains of 3-input max.
 __device__ __forceinline__ float max64(const float (&v)[64]) {
@@ -160,8 +180,11 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* turn = o_free + 2;               // [2] softmax ping-pong (4 warp arrivals)
     uint64_t* drain = turn + 2;                // [2]
     uint64_t* p_half = drain + 2;              // [2] first half of P_t written (4 warp arrivals)
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(p_half + 2);
+    uint64_t* item_full = p_half + 2;          // [ITEM_RING] work item r published
+    uint64_t* item_empty = item_full + C::ITEM_RING;  // [ITEM_RING] read by every role (ITEM_READERS arrivals)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(item_empty + C::ITEM_RING);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    volatile int* item_ring = reinterpret_cast<volatile int*>(tmem_holder + 4);  // [ITEM_RING]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -181,6 +204,10 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&slot_full[i], C::CHUNKS);
             mbar_init(&slot_empty[i], 2);  // released by both query tiles' MMAs
         }
+        for (int i = 0; i < C::ITEM_RING; ++i) {
+            mbar_init(&item_full[i], 1);
+            mbar_init(&item_empty[i], C::ITEM_READERS);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -192,6 +219,38 @@ __global__ void __launch_bounds__(384, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+
+    // Work item r of this CTA: published by the first producer's thread (the
+    // first item is the CTA's index, later ones come from the launch's counter,
+    // taken while the previous item's last loads are issued so that the atomic's
+    // latency hides behind them; p.n_items marks the end), read by every other
+    // role in the same order. Returns the item, or -1 when a wait was abandoned.
+    auto take_item = [&]() -> int {
+        return static_cast<int>(gridDim.x + atomicAdd(&g_fwd_sched[p.sched_slot][0], 1u));
+    };
+    auto publish_item = [&](int r, int w) -> int {
+        const int s = r % C::ITEM_RING;
+        if (r >= C::ITEM_RING && !mbar_wait(&item_empty[s], ((r / C::ITEM_RING) - 1) & 1, abort_flag)) return -1;
+        if (w > p.n_items) w = p.n_items;
+        item_ring[s] = w;
+        mbar_arrive(&item_full[s]);
+        return w;
+    };
+    auto read_item = [&](int r) -> int {  // one thread: the second producer, an MMA issuer
+        const int s = r % C::ITEM_RING;
+        if (!mbar_wait(&item_full[s], (r / C::ITEM_RING) & 1, abort_flag)) return -1;
+        const int w = item_ring[s];
+        mbar_arrive(&item_empty[s]);
+        return w;
+    };
+    auto read_item_warp = [&](int r) -> int {  // all 32 lanes of a softmax warp
+        const int s = r % C::ITEM_RING;
+        const bool ok_w = mbar_wait(&item_full[s], (r / C::ITEM_RING) & 1, abort_flag);
+        const int w = item_ring[s];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&item_empty[s]);
+        return __all_sync(0xffffffffu, ok_w) ? w : -1;
+    };
 
     if (warp >= 10) {
         // ------------------------------------------------------ producers ---
@@ -206,8 +265,10 @@ __global__ void __launch_bounds__(384, 1)
             tma_prefetch_desc(&tm_v);
             bool ok = true;
             int g = 0, it = 0;
+            int next_w = static_cast<int>(blockIdx.x);  // first producer: the item it publishes next
             for (int r = 0; ok; ++r, ++it) {
-                const int w = fwd_work_index(r);
+                const int w = CAUSAL ? fwd_work_index(r) : me == 0 ? publish_item(r, next_w) : read_item(r);
+                if (w < 0) { ok = false; break; }
                 if (w >= p.n_items) break;
                 const FwdItem item = fwd_item<CAUSAL>(p, w);
                 const int zq = item.b * p.Hq + item.h, zkv = item.b * p.Hkv + item.hk;
@@ -250,8 +311,19 @@ __global__ void __launch_bounds__(384, 1)
                 // item), K_0 and V_0 (slots the previous item's last tiles release),
                 // then Q tile 1 (free after tile 1's last S, one key tile later in a
                 // causal item), then the rest.
+                // the first producer takes the next item two key tiles before this
+                // item's last loads
+                const int take_at = max(2, 2 * item.nk1 - 4);
+                bool taken = false;
                 ok = issue_q(0) && issue_kv(0) && issue_kv(1) && issue_q(1);
-                for (int i = 2; ok && i < 2 * item.nk1; ++i) ok = issue_kv(i);
+                for (int i = 2; ok && i < 2 * item.nk1; ++i) {
+                    if (!CAUSAL && me == 0 && i == take_at) {
+                        next_w = take_item();
+                        taken = true;
+                    }
+                    ok = issue_kv(i);
+                }
+                if (!CAUSAL && me == 0 && !taken) next_w = take_item();
                 g += 2 * item.nk1;
             }
             // Let every copy in flight land before the CTA can exit.
@@ -273,7 +345,8 @@ __global__ void __launch_bounds__(384, 1)
             int g = 0;        // K/V load index of the item's K_0
             uint32_t np = 0;  // P_t handed over so far (p_full phases)
             for (int r = 0, it = 0; ok; ++r, ++it) {
-                const int w = fwd_work_index(r);
+                const int w = CAUSAL ? fwd_work_index(r) : read_item(r);
+                if (w < 0) { ok = false; break; }
                 if (w >= p.n_items) break;
                 const FwdItem item = fwd_item<CAUSAL>(p, w);
                 const int nk = t ? item.nk1 : item.nk0;
@@ -356,10 +429,10 @@ __global__ void __launch_bounds__(384, 1)
         bool ok = true;
         uint32_t ns = 0, nturn = 0, npv = 0;  // phases consumed so far, counted across items
         for (int r = 0; ok; ++r) {
-            const int w = fwd_work_index(r);
+            const int w = CAUSAL ? fwd_work_index(r) : read_item_warp(r);
+            if (w < 0) { ok = false; break; }
             if (w >= p.n_items) break;
             const FwdItem item = fwd_item<CAUSAL>(p, w);
-            const bool has_next = fwd_work_index(r + 1) < p.n_items;
             const int nk = t ? item.nk1 : item.nk0;
             const int grow = item.qb * 2 * BM + t * BM + row;
             const int q128 = 2 * item.qb + t;  // index of this query tile in 128-row units
@@ -458,9 +531,9 @@ __global__ void __launch_bounds__(384, 1)
                 l += rs.x + rs.y;
                 // pass the turn on: tile 0 always hands over to tile 1 of the same key
                 // tile; tile 1 hands back after each key tile it shares with tile 0
-                // (for key tile j + 1 of this item, or key tile 0 of the next item)
-                const bool hand_over =
-                    (t == 0) || (j + 1 < item.nk0) || (j == item.nk0 - 1 && has_next);
+                // (for key tile j + 1 of this item, or key tile 0 of the next item;
+                // after the CTA's last item nobody waits for that turn)
+                const bool hand_over = (t == 0) || (j < item.nk0);
                 if (hand_over && lane == 0) mbar_arrive(&turn[1 - t]);
                 tmem_st_wait();
                 tc_fence_before();
@@ -559,6 +632,16 @@ __global__ void __launch_bounds__(384, 1)
     if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+    // Every item this CTA took has been taken; the last CTA to get here resets the
+    // launch's counter slot (no CTA of this launch reads it any more).
+    if (!CAUSAL && threadIdx.x == 0) {
+        unsigned int* ctr = g_fwd_sched[p.sched_slot];
+        __threadfence();
+        if (atomicAdd(&ctr[1], 1u) == gridDim.x - 1) {
+            atomicExch(&ctr[0], 0u);
+            atomicExch(&ctr[1], 0u);
+        }
     }
 }
 

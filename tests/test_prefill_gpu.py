@@ -180,3 +180,48 @@ def test_repeatable_large_logits_many_tiles():
     for _ in range(3):
         o2, l2 = run_gpu(q, k, v, False, 128 ** -0.5)
         assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_work_counter_slots_are_reused_and_reset():
+    """Non-causal launches hand out work items from a per-launch counter slot
+    that the launch's last CTA resets. 70 launches in a row (more than the 64
+    slots, so slots are used twice) on a problem with more items than CTAs, each
+    into a NaN-poisoned output, all give the first launch's result bit for bit:
+    every item is computed once by one CTA whichever CTA takes it."""
+    B, H, N, d = 2, 32, 1024, 128  # 4 query blocks x 64 planes = 256 items > 148 CTAs
+    q, k, v = (t.to(DEV) for t in si.make_qkv(6100, B, H, H, N, d))
+    refs = {c: eab.attention(q, k, v, causal=c) for c in (False, True)}
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, N, device=DEV)
+    for i in range(70):
+        causal = i % 5 == 4  # mostly non-causal launches, which take items from the counter
+        o.fill_(float("nan"))
+        lse.fill_(float("nan"))
+        eab.attn_fwd(q, k, v, o, lse, causal, d ** -0.5)
+        torch.cuda.synchronize()
+        assert torch.equal(o, refs[causal][0]) and torch.equal(lse, refs[causal][1]), f"launch {i}"
+    assert eab.attn_device_status() == 0
+
+
+def test_concurrent_launches_on_two_streams():
+    """Launches in flight at the same time on two streams take different counter
+    slots and do not steal each other's work items."""
+    B, H, N, d = 2, 32, 1536, 128
+    q, k, v = (t.to(DEV) for t in si.make_qkv(6200, B, H, H, N, d))
+    ref_c = eab.attention(q, k, v, causal=True)
+    ref_n = eab.attention(q, k, v, causal=False)
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    outs = []
+    for i in range(8):
+        oc, lc = torch.full_like(q, float("nan")), torch.full((B, H, N), float("nan"), device=DEV)
+        on, ln = torch.full_like(q, float("nan")), torch.full((B, H, N), float("nan"), device=DEV)
+        torch.cuda.synchronize()
+        eab.attn_fwd(q, k, v, oc, lc, True, d ** -0.5, s1)
+        eab.attn_fwd(q, k, v, on, ln, False, d ** -0.5, s2)
+        outs.append((oc, lc, on, ln))
+    torch.cuda.synchronize()
+    assert eab.attn_device_status() == 0
+    for oc, lc, on, ln in outs:
+        assert torch.equal(oc, ref_c[0]) and torch.equal(lc, ref_c[1])
+        assert torch.equal(on, ref_n[0]) and torch.equal(ln, ref_n[1])
