@@ -71,8 +71,8 @@ NCU_TRAFFIC = {
     "decode": {"bytes_per_launch": 536989440 + 3163904, "source_sha": "e8f2cefbecba28e0"},
     "decode_b1_l32k": {"bytes_per_launch": 134306560 + 3091456, "source_sha": "e8f2cefbecba28e0"},
     "decode_b8_l32k": {"bytes_per_launch": 1074017280 + 3969536, "source_sha": "e8f2cefbecba28e0"},
-    "attn_fwd_causal": {"bytes_per_launch": 144750080 + 15959552, "source_sha": "410f38f5c06bc391"},
-    "attn_fwd_noncausal": {"bytes_per_launch": 100970496 + 10457344, "source_sha": "410f38f5c06bc391"},
+    "attn_fwd_causal": {"bytes_per_launch": 141846528 + 15796480, "source_sha": "fbfe229d8b179eb0"},
+    "attn_fwd_noncausal": {"bytes_per_launch": 100948992 + 11680256, "source_sha": "fbfe229d8b179eb0"},
 }
 
 
@@ -431,7 +431,7 @@ def run_ours(args):
                              "launches": "bwd_delta_kernel, bwd_tile_kernel dK/dV, bwd_tile_kernel dQ"},
                 "fp8_forward": {"ms": round(t_fp8, 5), "tflops": round(p.flops() / (t_fp8 * 1e-3) / 1e12, 1),
                                 "peak": round(2 * tc_peak, 1),
-                                "peak_source": "measured bf16_tflops x 2 (nominal fp8 / bf16 ratio)",
+                                "peak_source": f"{peak_src} bf16_tflops x 2 (nominal fp8 / bf16 ratio)",
                                 "frac": round(p.flops() / (t_fp8 * 1e-3) / 1e12 / (2 * tc_peak), 4),
                                 "quant_ms_q_k_v": round(t_quant, 5)},
             }

@@ -421,11 +421,23 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, cons
     p.lse = lse;
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.nblk = nblk;
     p.scale_log2 = scale * kLog2e;
+    p.n_qblocks = (N + 255) / 256;
+    const long long items = static_cast<long long>(p.n_qblocks) * B * Hq;
+    if (items > (1LL << 30)) return ATTN_ERR_INVALID_ARG;
+    p.n_items = static_cast<int>(items);
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        return ATTN_ERR_CUDA;
+    // without the causal mask a grid of up to twice the items lets the kernel
+    // deal 128-row halves to otherwise idle SMs
+    const int want = (!causal && 2 * p.n_items <= sms) ? 2 * p.n_items : p.n_items;
+    const int grid = want < sms ? want : sms;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     auto kern = causal ? attn_fwd_fp8_kernel<true> : attn_fwd_fp8_kernel<false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Fp8Cfg::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
-    kern<<<dim3(nblk, B * Hq), Fp8Cfg::NUM_THREADS, Fp8Cfg::SMEM_BYTES, st>>>(tq, tk, tv, p);
+    kern<<<grid, Fp8Cfg::NUM_THREADS, Fp8Cfg::SMEM_BYTES, st>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -315,6 +315,28 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
     return d;
 }
 
+// 2^y for a pair of values on the FMA and integer pipes instead of the MUFU
+// (Cody-Waite style range reduction plus a polynomial): y = j + r with
+// j = rint(y), taken with the 1.5 * 2^23 shifter, and r in [-1/2, 1/2]; 2^r
+// from the degree-3 polynomial with p(0) = 1 that minimises the largest
+// relative error on that interval (fit_exp2_poly.py: 1.0e-4, a twentieth of a
+// bf16 half-ulp); 2^j added into the exponent field. y is clamped to >= -126,
+// so the result is >= 0 and below 2^-125 there: callers that need an exact 0
+// (masked scores) use ex2_approx instead.
+__device__ __forceinline__ float2 exp2_poly3x2(float2 y) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    y = make_float2(fmaxf(y.x, -126.f), fmaxf(y.y, -126.f));
+    const float2 t = fadd2(y, make_float2(kShift, kShift));
+    const float2 jf = fadd2(t, make_float2(-kShift, -kShift));
+    const float2 r = fadd2(y, make_float2(-jf.x, -jf.y));
+    float2 p = ffma2(r, make_float2(0x1.c2a25cp-5f, 0x1.c2a25cp-5f), make_float2(0x1.f00c4ep-3f, 0x1.f00c4ep-3f));
+    p = ffma2(p, r, make_float2(0x1.62f5fap-1f, 0x1.62f5fap-1f));
+    p = ffma2(p, r, make_float2(1.f, 1.f));
+    // the low bits of t hold j in two's complement: t << 23 is j << 23
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
