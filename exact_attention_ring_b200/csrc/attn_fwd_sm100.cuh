@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(384, 1)
                     for (int c = 0; c < C::CHUNKS; ++c) mine |= ((gi * C::CHUNKS + c) % C::NUM_PRODUCERS) == me;
                     if (!mine) return true;
                     const int slot = gi % SLOTS, use = gi / SLOTS;
-                    if (use > 0 && !mbar_wait(&slot_empty[slot], (use - 1) & 1, abort_flag)) return false;
+                    if (use > 0 && !mbar_wait_park(&slot_empty[slot], (use - 1) & 1, abort_flag)) return false;
                     const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;
                     uint8_t* dst = sKV + slot * C::TILE_BYTES;
 #pragma unroll
@@ -297,7 +297,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                     for (int c = 0; c < C::CHUNKS; ++c) any |= ((t * C::CHUNKS + c) % C::NUM_PRODUCERS) == me;
                     if (!any) return true;
-                    if (it > 0 && !mbar_wait(&q_empty[t], (it - 1) & 1, abort_flag)) return false;
+                    if (it > 0 && !mbar_wait_park(&q_empty[t], (it - 1) & 1, abort_flag)) return false;
 #pragma unroll
                     for (int c = 0; c < C::CHUNKS; ++c) {
                         if ((t * C::CHUNKS + c) % C::NUM_PRODUCERS != me) continue;

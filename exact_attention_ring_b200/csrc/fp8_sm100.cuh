@@ -467,7 +467,7 @@ __global__ void __launch_bounds__(384, 1)
                     const int gi = g + i;
                     if ((gi & 1) != me) return true;
                     const int slot = gi % SLOTS, use = gi / SLOTS;
-                    if (use > 0 && !mbar_wait(&slot_empty[slot], (use - 1) & 1, abort_flag)) return false;
+                    if (use > 0 && !mbar_wait_park(&slot_empty[slot], (use - 1) & 1, abort_flag)) return false;
                     mbar_arrive_expect_tx(&slot_full[slot], TILE);
                     if (i & 1) tma_load_3d(sKV + slot * TILE, &tm_vt, &slot_full[slot], (i >> 1) * BN, 0, zkv);
                     else tma_load_3d(sKV + slot * TILE, &tm_k, &slot_full[slot], 0, (i >> 1) * BN, zkv);
@@ -475,7 +475,7 @@ __global__ void __launch_bounds__(384, 1)
                 };
                 auto issue_q = [&](int t) -> bool {
                     if ((t & 1) != me || (t == 1 && item.nk1 == 0)) return true;
-                    if (nq[t] > 0 && !mbar_wait(&q_empty[t], (nq[t] - 1) & 1, abort_flag)) return false;
+                    if (nq[t] > 0 && !mbar_wait_park(&q_empty[t], (nq[t] - 1) & 1, abort_flag)) return false;
                     mbar_arrive_expect_tx(&q_full[t], TILE);
                     tma_load_3d(sQ + t * TILE, &tm_q, &q_full[t], 0, (item.q0 + t) * BM, zq);
                     ++nq[t];

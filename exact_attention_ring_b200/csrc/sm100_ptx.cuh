@@ -99,6 +99,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     return mbar_wait_slow(bar, parity, abort, limit_ns);
 }
 
+// Waits by suspending probes only (try_wait parks the thread until the phase
+// completes or a short system time limit passes), for long waits off the
+// critical path, such as a producer waiting for a ring slot: the waiter takes
+// no issue slots from the warps that share its sub-partition, at the price of
+// waking a few hundred cycles late.
+__device__ __forceinline__ bool mbar_wait_park(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+#pragma unroll 1
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (abort != nullptr && *abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            atomicCAS(&g_attn_status, 0, kStatusTimeout);
+            if (abort != nullptr) *abort = 1;
+            return false;
+        }
+    }
+}
+
 // Waits by non-blocking probes only (no suspended try_wait), for the waits on
 // the critical path of a waiter that has nothing else to do.
 __device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort,
