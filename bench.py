@@ -7,8 +7,11 @@ One step is one pass of the whole path over one batch of synthetic inputs:
   2. attn_fwd, non-causal, same shape
   3. attn_decode_splitkv + 4. attn_combine on single-query decode
      (B=1, Hq=32, Hkv=8, L=131072, d=128; the default split count).
-After the timed loop the same decode pair at L=32768 for B=1 and B=8 is timed
-alone (L2 flushed before every launch) and reported beside the step's kernels.
+The decode pair is timed as one interval (the combine is launched with
+programmatic stream serialization, so its launch overlaps the decode's end).
+After the timed loop every decode kernel is also timed alone, and the same
+pair at L=32768 for B=1 and B=8 (L2 flushed before every launch); both are
+reported beside the step's kernels.
 The printed `value` is the causal prefill's TFLOPS (4*B*H*N^2*d/2 per launch
 over the kernel's CUDA-event time, summed over all ranks); the decode's KV-read
 GB/s is reported beside it. Inputs are seeded N(0,1) bf16, resident in HBM
@@ -68,12 +71,11 @@ NCU_TRAFFIC = {
     # L32768 decodes; attn_fwd_kernel<128, causal / non-causal>: B2 H32 N2048 d128. Read + write
     # with cold caches (ncu flushes them before each captured launch); the prefill's O (33.5 MB)
     # mostly stays dirty in L2 when the kernel ends, so its write-back is not counted here.
-    "decode": {"bytes_per_launch": 536989440 + 3163904, "source_sha": "e8f2cefbecba28e0"},
-    "decode_b1_l32k": {"bytes_per_launch": 134306560 + 3091456, "source_sha": "e8f2cefbecba28e0"},
-    "decode_b8_l32k": {"bytes_per_launch": 1074017280 + 3969536, "source_sha": "e8f2cefbecba28e0"},
-    "attn_fwd_causal": {"bytes_per_launch": 141846528 + 15796480, "source_sha": "fbfe229d8b179eb0"},
-    "attn_fwd_noncausal": {"bytes_per_launch": 100948992 + 11680256, "source_sha": "fbfe229d8b179eb0"},
-}
+    "decode": {"bytes_per_launch": 536959744 + 3461376, "source_sha": "eaaf414296e5590d"},
+    "decode_b1_l32k": {"bytes_per_launch": 134302976 + 3129856, "source_sha": "eaaf414296e5590d"},
+    "decode_b8_l32k": {"bytes_per_launch": 1073927168 + 3971072, "source_sha": "eaaf414296e5590d"},
+    "attn_fwd_causal": {"bytes_per_launch": 135838720 + 15925760, "source_sha": "462252897f7ebb02"},
+    "attn_fwd_noncausal": {"bytes_per_launch": 101012224 + 12996096, "source_sha": "462252897f7ebb02"},
 
 
 def kernel_sha(name: str) -> str:
@@ -257,21 +259,32 @@ def run_ours(args):
     flush_read = torch.ones(2 * L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32)  # 512 MB
     flush_sum = torch.empty((), device=dev, dtype=torch.float32)
 
-    n_ev = 5
+    n_ev = 4
     def flush_l2():
         # write a buffer larger than L2, then read another: the next kernel starts
         # with none of its inputs in L2 and no dirty lines to write back
         flush.fill_(float(rank))
         torch.sum(flush_read, dim=0, out=flush_sum)
 
-    def run_decode(ds, ev=None, i0=0):
+    def run_decode(ds, combine=True):
+        # the pair back to back: the combine is launched with programmatic stream
+        # serialization, so its launch overlaps the decode's last blocks
         eab.attn_decode_splitkv(ds["q"], ds["k"], ds["v"], ds["o_part"], ds["lse_part"], ds["S"],
                                 ds["shape"].scale, stream)
-        if ev is not None:
-            ev[i0].record(stream)
-        eab.attn_combine(ds["o_part"], ds["lse_part"], ds["o"], ds["lse"], stream)
-        if ev is not None:
-            ev[i0 + 1].record(stream)
+        if combine:
+            eab.attn_combine(ds["o_part"], ds["lse_part"], ds["o"], ds["lse"], stream)
+
+    def median_ms(fn, n=10):
+        # n launches of fn, each after a flush, timed alone: the median (every rank
+        # runs the same launches)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+        for a, b in evs:
+            flush_l2()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in evs), world)
 
     def step(ev=None):
         if ev is not None:
@@ -282,7 +295,9 @@ def run_ours(args):
         eab.attn_fwd(q, k, v, o2, lse2, False, p.scale, stream)
         if ev is not None:
             ev[2].record(stream)
-        run_decode(dec_sets[0], ev, 3)
+        run_decode(dec_sets[0])
+        if ev is not None:
+            ev[3].record(stream)
         flush_l2()
 
     for _ in range(args.warmup):
@@ -305,29 +320,24 @@ def run_ours(args):
     t_fwd_c = sum(e[0].elapsed_time(e[1]) for e in events) / args.steps
     t_fwd_n = sum(e[1].elapsed_time(e[2]) for e in events) / args.steps
     t_fwd_c, t_fwd_n = (max_over_ranks(x, world) for x in (t_fwd_c, t_fwd_n))
-    dec_sets[0]["t_dec"] = max_over_ranks(sum(e[2].elapsed_time(e[3]) for e in events) / args.steps, world)
-    dec_sets[0]["t_comb"] = max_over_ranks(sum(e[3].elapsed_time(e[4]) for e in events) / args.steps, world)
-    t_dec, t_comb = dec_sets[0]["t_dec"], dec_sets[0]["t_comb"]
-    # the L = 32768 decodes, timed alone after the loop: median of 10 launches, each
-    # after a flush (every rank runs the same launches)
-    for ds in dec_sets[1:]:
+    # the step's decode + combine, as one interval (the metric's time)
+    dec_sets[0]["t_pair"] = max_over_ranks(sum(e[2].elapsed_time(e[3]) for e in events) / args.steps, world)
+    # after the loop: every decode kernel alone (for its roofline), and the L = 32768
+    # decode + combine pairs; median of 10 launches, each after a flush
+    for ds in dec_sets:
         for _ in range(3):
             run_decode(ds)
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(10)]
-        for ev3 in evs:
-            flush_l2()
-            ev3[0].record(stream)
-            run_decode(ds, ev3, 1)
-        torch.cuda.synchronize()
-        ds["t_dec"] = max_over_ranks(statistics.median(e[0].elapsed_time(e[1]) for e in evs), world)
-        ds["t_comb"] = max_over_ranks(statistics.median(e[1].elapsed_time(e[2]) for e in evs), world)
+        ds["t_dec"] = median_ms(lambda: run_decode(ds, combine=False))
+        if ds is not dec_sets[0]:
+            ds["t_pair"] = median_ms(lambda: run_decode(ds))
+    t_dec, t_pair = dec_sets[0]["t_dec"], dec_sets[0]["t_pair"]
     assert eab.attn_device_status() == 0
     assert eab.attn_device_status() == 0
 
     tflops_c = p.flops() / (t_fwd_c * 1e-3) / 1e12
     tflops_n = PREFILL_NC.flops() / (t_fwd_n * 1e-3) / 1e12
     kv_bytes = dc.kv_bytes()
-    dec_gbs = kv_bytes / ((t_dec + t_comb) * 1e-3) / 1e9
+    dec_gbs = kv_bytes / (t_pair * 1e-3) / 1e9
     dec_kernel_gbs = kv_bytes / (t_dec * 1e-3) / 1e9
 
     # ---- end to end through the public API with host buffers (causal prefill).
@@ -405,15 +415,18 @@ def run_ours(args):
         dec_roofs[ds["name"]] = {
             "kernel": "decode_splitkv_keys_kernel<16,3> (keys as tile rows)", "bound": "hbm", "achieved": round(gbs, 1),
             "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4),
-            "traffic": traffic(ds["name"], dec_sha), "ms": round(ds["t_dec"], 5), "ms_combine": round(ds["t_comb"], 5),
-            "with_combine_gbs": round(shp.kv_bytes() / ((ds["t_dec"] + ds["t_comb"]) * 1e-3) / 1e9, 1),
+            "traffic": traffic(ds["name"], dec_sha), "ms": round(ds["t_dec"], 5),
+            "ms_with_combine": round(ds["t_pair"], 5),
+            "with_combine_gbs": round(shp.kv_bytes() / (ds["t_pair"] * 1e-3) / 1e9, 1),
             "workload": f"B{shp.B} Hq{shp.Hq} Hkv{shp.Hkv} L{shp.L} d{shp.d}, {ds['S']} splits",
             "peak_source": f"{peak_src} hbm_gbs"}
     roof_dec = dec_roofs["decode"]
-    for ds in dec_sets[1:]:
-        dec_roofs[ds["name"]]["timed"] = "alone after the step loop, L2 flushed before each launch, median of 10"
+    for ds in dec_sets:
+        dec_roofs[ds["name"]]["timed"] = ("kernel alone after the step loop, L2 flushed before each launch, median "
+                                          "of 10; with the combine: " + ("the step's interval" if ds is dec_sets[0]
+                                                                         else "the same, the pair back to back"))
     # the dominant kernel: the one that takes the most time in the step
-    times = {"fwd_causal": t_fwd_c, "fwd_noncausal": t_fwd_n, "decode": t_dec}
+    times = {"fwd_causal": t_fwd_c, "fwd_noncausal": t_fwd_n, "decode": t_pair}
     dominant = max(times, key=times.get)
     roofline = {"fwd_causal": roof_fwd, "fwd_noncausal": roof_fwd_nc, "decode": roof_dec}[dominant]
 
@@ -467,7 +480,9 @@ def run_ours(args):
             },
             "decode": {"value": round(dec_gbs * world, 1), "unit": "GB/s", "kernel_gbs": round(dec_kernel_gbs, 1),
                        "frac_hbm": round(dec_kernel_gbs / hbm_peak, 4), "ms_decode": round(t_dec, 5),
-                       "ms_combine": round(t_comb, 5), "kv_bytes": kv_bytes},
+                       "ms_decode_and_combine": round(t_pair, 5), "kv_bytes": kv_bytes,
+                       "timing": "value: the step's decode + combine as one event interval; kernel_gbs: the "
+                                 "decode kernel alone after the loop (flushed L2, median of 10)"},
             "prefill_noncausal": {"value": round(tflops_n * world, 2), "unit": "TFLOPS",
                                   "frac": round(tflops_n / tc_peak, 4)},
             "roofline": roofline,

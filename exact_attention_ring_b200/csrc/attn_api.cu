@@ -10,6 +10,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <utility>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -23,6 +24,28 @@
 
 namespace eab {
 namespace {
+
+// Launch with programmatic stream serialization: the kernel's blocks may be
+// scheduled while the previous kernel in the stream is finishing (once all of
+// its blocks have issued griddepcontrol.launch_dependents or exited); every
+// kernel launched this way calls grid_dep_wait() before its first global
+// memory access, so the order of the stream's memory effects is unchanged.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -98,7 +121,8 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
         return ATTN_ERR_CUDA;
     const int grid = p.n_items < sms ? p.n_items : sms;
-    kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    if (launch_pdl(kern, dim3(grid), dim3(C::NUM_THREADS), C::SMEM_BYTES, stream, tq, tk, tv, p) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -109,7 +133,8 @@ attn_status_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const 
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
     const dim3 grid(p.S, p.Hkv * p.groups, p.B);
-    kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
+    if (launch_pdl(kern, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, stream, tk, tv, p) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -123,7 +148,8 @@ attn_status_t launch_decode_keys(const CUtensorMap& tk, const CUtensorMap& tv, c
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
     const dim3 grid(p.S, p.Hkv, p.B);
-    kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
+    if (launch_pdl(kern, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, stream, tk, tv, p) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -178,7 +204,8 @@ attn_status_t launch_bwd_tile(const CUtensorMap& fa, const CUtensorMap& fb, cons
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
     const dim3 grid((p.N + C::BT - 1) / C::BT, p.B * (DKDV ? p.Hkv : p.Hq));
-    kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(fa, fb, sa, sb, p);
+    if (launch_pdl(kern, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, stream, fa, fb, sa, sb, p) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -186,7 +213,7 @@ template <int D, bool CAUSAL>
 attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
     const long long rows = static_cast<long long>(p.B) * p.Hq * p.N;
-    bwd_delta_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p, rows);
+    launch_pdl(bwd_delta_kernel<D>, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, stream, p, rows);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     attn_status_t st = launch_bwd_tile<D, CAUSAL, true>(tk, tv, tq, tdo, p, stream);
     if (st != ATTN_OK) return st;
@@ -237,9 +264,11 @@ attn_status_t combine_impl(const float* o_part, const float* lse_part, void* o, 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     auto* ob = static_cast<typename E::T*>(o);
     if (d == 128)
-        combine_kernel<128, E><<<static_cast<unsigned>(blocks), 128, smem, st>>>(o_part, lse_part, ob, lse, num_splits);
+        launch_pdl(combine_kernel<128, E>, dim3(static_cast<unsigned>(blocks)), dim3(128), smem, st, o_part, lse_part,
+                   ob, lse, num_splits);
     else
-        combine_kernel<64, E><<<static_cast<unsigned>(blocks), 64, smem, st>>>(o_part, lse_part, ob, lse, num_splits);
+        launch_pdl(combine_kernel<64, E>, dim3(static_cast<unsigned>(blocks)), dim3(64), smem, st, o_part, lse_part,
+                   ob, lse, num_splits);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -309,9 +338,11 @@ attn_status_t attn_merge(float* o_acc, float* lse_acc, const float* o_blk, const
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     auto* outb = static_cast<__nv_bfloat16*>(out);
     if (d == 128)
-        merge_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(o_acc, lse_acc, o_blk, lse_blk, outb, rows, init);
+        launch_pdl(merge_kernel<128>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, o_acc, lse_acc, o_blk,
+                   lse_blk, outb, rows, init);
     else
-        merge_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(o_acc, lse_acc, o_blk, lse_blk, outb, rows, init);
+        launch_pdl(merge_kernel<64>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, o_acc, lse_acc, o_blk,
+                   lse_blk, outb, rows, init);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -363,20 +394,20 @@ attn_status_t attn_quant_fp8(const void* x, void* codes, float* scales, int plan
     const dim3 grid(nblk, planes);
     if (!per_plane && !transpose) {
         // per-block scales, row-major codes: one pass over x
-        if (d == 128) fp8_quant_rows_kernel<128, false><<<grid, 256, 0, st>>>(p);
-        else fp8_quant_rows_kernel<64, false><<<grid, 256, 0, st>>>(p);
+        if (d == 128) launch_pdl(fp8_quant_rows_kernel<128, false>, grid, dim3(256), 0, st, p);
+        else launch_pdl(fp8_quant_rows_kernel<64, false>, grid, dim3(256), 0, st, p);
         return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
     }
     if (d == 128) {
-        fp8_amax_kernel<128><<<grid, 256, 0, st>>>(p);
-        if (transpose) fp8_quant_kernel<128, true><<<grid, 256, 0, st>>>(p);
-        else fp8_quant_kernel<128, false><<<grid, 256, 0, st>>>(p);
+        launch_pdl(fp8_amax_kernel<128>, grid, dim3(256), 0, st, p);
+        if (transpose) launch_pdl(fp8_quant_kernel<128, true>, grid, dim3(256), 0, st, p);
+        else launch_pdl(fp8_quant_kernel<128, false>, grid, dim3(256), 0, st, p);
     } else {
-        fp8_amax_kernel<64><<<grid, 256, 0, st>>>(p);
-        if (transpose) fp8_quant_kernel<64, true><<<grid, 256, 0, st>>>(p);
-        else fp8_quant_kernel<64, false><<<grid, 256, 0, st>>>(p);
+        launch_pdl(fp8_amax_kernel<64>, grid, dim3(256), 0, st, p);
+        if (transpose) launch_pdl(fp8_quant_kernel<64, true>, grid, dim3(256), 0, st, p);
+        else launch_pdl(fp8_quant_kernel<64, false>, grid, dim3(256), 0, st, p);
     }
-    fp8_scales_kernel<<<(planes + 255) / 256, 256, 0, st>>>(p);
+    launch_pdl(fp8_scales_kernel, dim3((planes + 255) / 256), dim3(256), 0, st, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -395,8 +426,8 @@ attn_status_t attn_quant_fp8_rotate(const void* x, const float* signs, void* cod
     p.rot_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const dim3 grid(nblk, planes);
-    if (d == 128) fp8_quant_rows_kernel<128, true><<<grid, 256, 0, st>>>(p);
-    else fp8_quant_rows_kernel<64, true><<<grid, 256, 0, st>>>(p);
+    if (d == 128) launch_pdl(fp8_quant_rows_kernel<128, true>, grid, dim3(256), 0, st, p);
+    else launch_pdl(fp8_quant_rows_kernel<64, true>, grid, dim3(256), 0, st, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -437,7 +468,8 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, cons
     auto kern = causal ? attn_fwd_fp8_kernel<true> : attn_fwd_fp8_kernel<false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Fp8Cfg::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
-    kern<<<grid, Fp8Cfg::NUM_THREADS, Fp8Cfg::SMEM_BYTES, st>>>(tq, tk, tv, p);
+    if (launch_pdl(kern, dim3(grid), dim3(Fp8Cfg::NUM_THREADS), Fp8Cfg::SMEM_BYTES, st, tq, tk, tv, p) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -219,6 +219,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    grid_dep_wait();  // the previous kernel's writes are visible from here on
 
     // Work item r of this CTA: published by the first producer's thread (the
     // first item is the CTA's index, later ones come from the launch's counter,
@@ -326,6 +327,9 @@ __global__ void __launch_bounds__(384, 1)
                 if (!CAUSAL && me == 0 && !taken) next_w = take_item();
                 g += 2 * item.nk1;
             }
+            // Every load of this CTA is issued: the next kernel in the stream may be
+            // scheduled (it waits for this grid's completion before reading memory).
+            grid_dep_launch();
             // Let every copy in flight land before the CTA can exit.
             if (it > 0) {
                 mbar_wait(&q_full[0], (it - 1) & 1, nullptr);

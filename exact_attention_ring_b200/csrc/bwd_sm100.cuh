@@ -66,6 +66,8 @@ struct BwdCfg {
 // Delta_i = sum_t dO_it O_it, one warp per row.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdParams p, long long rows) {
+    grid_dep_wait();  // the previous kernel's writes are visible from here on
+    grid_dep_launch();
     const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     if (row >= rows) return;
     const int lane = threadIdx.x & 31;
@@ -159,6 +161,7 @@ __global__ void __launch_bounds__(192, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    grid_dep_wait();  // the previous kernel's writes are visible from here on
 
     // plane (batch * heads + head) and tile row of streamed step s
     auto step_src = [&](int s, int* plane, int* trow) {
@@ -199,6 +202,9 @@ __global__ void __launch_bounds__(192, 1)
                     tma_load_3d(dst + C::TILE_BYTES + c * BOX, &tm_sb, &st_full[bu], c * 64, trow, plane);
                 }
             }
+            // Every load of this CTA is issued: the next kernel in the stream may be
+            // scheduled (it waits for this grid's completion before reading memory).
+            grid_dep_launch();
             // Let every copy in flight land before the CTA can exit.
             mbar_wait(fix_full, 0, nullptr);
             for (int i = max(0, s - 2); i < s; ++i) mbar_wait(&st_full[i & 1], (i >> 1) & 1, nullptr);

@@ -126,6 +126,7 @@ __global__ void __launch_bounds__(224, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    grid_dep_wait();  // the previous kernel's writes are visible from here on
 
     if (warp >= 5) {
         // ------------------------------------------------------ producers ---
@@ -154,6 +155,9 @@ __global__ void __launch_bounds__(224, 1)
                 }
                 issued = i + 1;
             }
+            // Every load of this CTA is issued: the next kernel in the stream may be
+            // scheduled (it waits for this grid's completion before reading memory).
+            grid_dep_launch();
             // Let every copy in flight land before the CTA can exit.
             for (int i = max(0, issued - SLOTS); i < issued; ++i)
                 mbar_wait(&slot_full[i % SLOTS], (i / SLOTS) & 1, nullptr);
@@ -450,6 +454,7 @@ __global__ void __launch_bounds__(224, DecTCfg<NQ, SLOTS_>::BLOCKS_PER_SM)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    grid_dep_wait();  // the previous kernel's writes are visible from here on
 
     if (warp >= 5) {
         // ------------------------------------------------------ producers ---
@@ -478,6 +483,9 @@ __global__ void __launch_bounds__(224, DecTCfg<NQ, SLOTS_>::BLOCKS_PER_SM)
                 }
                 issued = i + 1;
             }
+            // Every load of this CTA is issued: the next kernel in the stream may be
+            // scheduled (it waits for this grid's completion before reading memory).
+            grid_dep_launch();
             // Let every copy in flight land before the CTA can exit.
             for (int i = max(0, issued - SLOTS); i < issued; ++i)
                 mbar_wait(&slot_full[i % SLOTS], (i / SLOTS) & 1, nullptr);
@@ -699,6 +707,8 @@ __global__ void __launch_bounds__(D)
     __shared__ float red[D / 32];
     __shared__ float bcast;
     const int bh = blockIdx.x, t = threadIdx.x;
+    grid_dep_wait();  // the partials of the decode before it are complete and visible
+    grid_dep_launch();
     const float* lp = lse_part + static_cast<size_t>(bh) * S;
 
     float M = -INFINITY;

@@ -78,6 +78,8 @@ struct QuantParams {
 // takes exactly the fp32 operations of the transform's definition, in its order.
 template <int D, bool ROTATE>
 __global__ void __launch_bounds__(256) fp8_quant_rows_kernel(const QuantParams p) {
+    grid_dep_wait();  // the previous kernel's writes are visible from here on
+    grid_dep_launch();
     constexpr int E = D / 32, RPW = 16;
     const int blk = blockIdx.x, plane = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -168,6 +170,8 @@ __global__ void __launch_bounds__(256) fp8_quant_rows_kernel(const QuantParams p
 
 template <int D>
 __global__ void __launch_bounds__(256) fp8_amax_kernel(const QuantParams p) {
+    grid_dep_wait();  // the previous kernel's writes are visible from here on
+    grid_dep_launch();
     const int blk = blockIdx.x, plane = blockIdx.y;
     const int r0 = blk * 128, rows = min(128, p.N - r0);
     const __nv_bfloat16* src = p.x + (static_cast<size_t>(plane) * p.N + r0) * D;
@@ -197,6 +201,8 @@ __device__ __forceinline__ float fp8_scale_of(float amax) { return amax > 0.f ? 
 
 template <int D, bool TRANSPOSE>
 __global__ void __launch_bounds__(256) fp8_quant_kernel(const QuantParams p) {
+    grid_dep_wait();  // the previous kernel's writes are visible from here on
+    grid_dep_launch();
     const int blk = blockIdx.x, plane = blockIdx.y;
     const int r0 = blk * 128, rows = min(128, p.N - r0);
     const float* mx = p.scales + static_cast<size_t>(plane) * p.nblk;
@@ -258,6 +264,8 @@ __global__ void __launch_bounds__(256) fp8_quant_kernel(const QuantParams p) {
 }
 
 __global__ void fp8_scales_kernel(const QuantParams p) {
+    grid_dep_wait();  // the previous kernel's writes are visible from here on
+    grid_dep_launch();
     const int plane = blockIdx.x * blockDim.x + threadIdx.x;
     if (plane >= p.planes) return;
     float* mx = p.scales + static_cast<size_t>(plane) * p.nblk;
@@ -447,6 +455,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    grid_dep_wait();  // the previous kernel's writes are visible from here on
 
     if (warp >= 10) {
         // ------------------------------------------------------ producers ---
@@ -485,6 +494,9 @@ __global__ void __launch_bounds__(384, 1)
                 for (int i = 2; ok && i < 2 * item.nkv; ++i) ok = issue_kv(i);
                 g += 2 * item.nkv;
             }
+            // Every load of this CTA is issued: the next kernel in the stream may be
+            // scheduled (it waits for this grid's completion before reading memory).
+            grid_dep_launch();
             // Let every copy in flight land before the CTA can exit.
             if (nq[me] > 0) mbar_wait(&q_full[me], (nq[me] - 1) & 1, nullptr);
             for (int i = max(0, g - SLOTS); i < g; ++i)

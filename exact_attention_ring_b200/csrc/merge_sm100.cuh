@@ -23,6 +23,8 @@ template <int D>
 __global__ void __launch_bounds__(256)
     merge_kernel(float* __restrict__ o_acc, float* __restrict__ lse_acc, const float* __restrict__ o_blk,
                  const float* __restrict__ lse_blk, __nv_bfloat16* __restrict__ out, long long rows, int init) {
+    grid_dep_wait();  // the previous kernel's writes are visible from here on
+    grid_dep_launch();
     constexpr int CPL = D / 32;  // columns per lane
     const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     if (row >= rows) return;

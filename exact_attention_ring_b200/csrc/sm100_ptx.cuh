@@ -292,6 +292,15 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Programmatic dependent launch. grid_dep_wait: returns once every grid this one
+// depends on (the previous kernel in the stream, when this one was launched
+// with programmatic stream serialization) has completed and its memory
+// operations are visible; at once otherwise. grid_dep_launch: this block no
+// longer holds back the launch of the next such kernel, which still waits for
+// this grid's completion before touching memory.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ math ----
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
