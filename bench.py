@@ -76,6 +76,7 @@ NCU_TRAFFIC = {
     "decode_b8_l32k": {"bytes_per_launch": 1073927168 + 3971072, "source_sha": "eaaf414296e5590d"},
     "attn_fwd_causal": {"bytes_per_launch": 135838720 + 15925760, "source_sha": "462252897f7ebb02"},
     "attn_fwd_noncausal": {"bytes_per_launch": 101012224 + 12996096, "source_sha": "462252897f7ebb02"},
+}
 
 
 def kernel_sha(name: str) -> str:
