@@ -24,12 +24,14 @@
 //                           dS (bf16) over dP, dQ += dS K (then times scale).
 // 192 threads each: warps 0-3 element-wise work and epilogue (thread = TMEM
 // lane), warp 4 the MMA issuer, warp 5 the TMA producer. Within a step the
-// element-wise pass computes P from S^T while dP^T is still being computed,
-// and hands P and dS over in two halves of 64 columns: the accumulating MMAs
-// of the first half run while the second half is computed. The next step's
-// S^T / dP^T MMAs are issued after the accumulating MMAs that read P^T / dS^T
-// from the same columns, so the tensor pipe's issue order keeps them intact
-// until read (as in the forward pass). Every wait is bounded.
+// element-wise pass reads S^T into registers at once, so the next step's S^T
+// MMAs run while it computes P (as dP^T is completing) and dS; P and dS go
+// back as bf16 over dP^T's columns, a quarter at a time, and are handed over
+// in two halves of 64 columns: the accumulating MMAs of the first half run
+// while the second half is computed. The next step's dP^T MMAs are issued
+// after the accumulating MMAs that read P^T / dS^T from its columns, so the
+// tensor pipe's issue order keeps them intact until read (as in the forward
+// pass). Every wait is bounded.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -86,14 +88,17 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdParams p, long 
 // tiles (A_fix, B_fix: K and V for dK/dV; Q and dO for dQ) and streams pairs of
 // tiles (S_a, S_b: Q and dO; K and V) through two buffers. Per step:
 //   X = A_fix S_a^T, then Y = B_fix S_b^T          (M = 128, N = 128, K = D)
-//   element-wise, in two halves of 64 columns:
-//     P = exp2(X scale log2e - lse log2e)  (while Y is still being computed),
-//     G = P o (Y - Delta), both written back as bf16 over X and Y
+//   element-wise: X into registers (X's columns are then free, and the MMA
+//     issuer starts X of the next step), P = exp2(X scale log2e - lse log2e)
+//     for the 128 columns, then per quarter of 32 columns G = P o (Y - Delta)
+//     with P and G written back as bf16 pairs over that quarter of Y
+//     (columns 32q .. 32q + 15 and 32q + 16 .. 32q + 31), announced per half
 //   acc1 += P S_b, acc2 += G S_a                    (A from TMEM, B MN-major)
 // The accumulating MMAs of the first half run while the second half is being
-// computed. For dQ only acc2 (dS K) is kept. scale multiplies acc2 once, in
-// the epilogue. Steps whose tile holds no masked element (off the causal
-// diagonal, inside the sequence) skip the mask.
+// computed; Y of the next step follows them. For dQ only acc2 (dS K) is kept
+// (P is not written back). scale multiplies acc2 once, in the epilogue. Steps
+// whose tile holds no masked element (off the causal diagonal, inside the
+// sequence) skip the mask.
 // TMEM: X [0, 128), Y [128, 256), acc1 [256, 256 + D), acc2 [256 + D, 256 + 2D).
 template <int D, bool CAUSAL, bool DKDV>
 __global__ void __launch_bounds__(192, 1)
@@ -119,7 +124,8 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* l_ready = bars + 9;    // [2] lse/Delta of a buffer staged (4 warp arrivals)
     uint64_t* l_free = bars + 11;    // [2] lse/Delta of a buffer read (4 warp arrivals)
     uint64_t* fin = bars + 13;       // every MMA done
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
+    uint64_t* x_read = bars + 14;    // X in the element-wise warps' registers (4 warp arrivals)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 15);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -150,6 +156,7 @@ __global__ void __launch_bounds__(192, 1)
         mbar_init(x_full, 1);
         mbar_init(y_full, 1);
         mbar_init(fin, 1);
+        mbar_init(x_read, 4);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -216,16 +223,12 @@ __global__ void __launch_bounds__(192, 1)
             constexpr uint32_t idesc_acc = make_idesc(BT, D, 0, 1, ElemBf16::fmt);  // B MN-major
             const uint32_t tX = tmem, tY = tmem + 128, tA1 = tmem + 256, tA2 = tmem + 256 + D;
             const uint32_t fa = smem_addr(sFA), fb = smem_addr(sFB);
-            bool ok = mbar_wait(fix_full, 0, abort_flag);
-            for (int s = 0; ok && s < nsteps; ++s) {
+            // X(s) = A_fix S_a(s)^T into X's columns, once step s's tiles have landed
+            auto issue_x = [&](int s) -> bool {
                 const int bu = s & 1;
-                const uint32_t sa = smem_addr(sS + bu * 2 * C::TILE_BYTES), sb = sa + C::TILE_BYTES;
-                ok = mbar_wait(&st_full[bu], (s >> 1) & 1, abort_flag);
-                if (!ok) break;
+                if (!mbar_wait(&st_full[bu], (s >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                // X = A_fix S_a^T, then Y = B_fix S_b^T. Issued after the previous
-                // step's accumulating MMAs, which read P and G from these columns:
-                // the tensor pipe's issue order keeps them intact until read.
+                const uint32_t sa = smem_addr(sS + bu * 2 * C::TILE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
@@ -233,6 +236,11 @@ __global__ void __launch_bounds__(192, 1)
                            kk > 0 ? 1u : 0u);
                 }
                 tc_commit(x_full);
+                return true;
+            };
+            // Y(s) = B_fix S_b(s)^T into Y's columns (after X(s): its tiles have landed)
+            auto issue_y = [&](int s) {
+                const uint32_t sb = smem_addr(sS + (s & 1) * 2 * C::TILE_BYTES) + C::TILE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
@@ -240,8 +248,22 @@ __global__ void __launch_bounds__(192, 1)
                            kk > 0 ? 1u : 0u);
                 }
                 tc_commit(y_full);
+            };
+            bool ok = mbar_wait(fix_full, 0, abort_flag) && issue_x(0);
+            if (ok) issue_y(0);
+            for (int s = 0; ok && s < nsteps; ++s) {
+                const int bu = s & 1;
+                const uint32_t sa = smem_addr(sS + bu * 2 * C::TILE_BYTES), sb = sa + C::TILE_BYTES;
+                // X(s+1) as soon as the element-wise warps hold X(s) in registers: it
+                // is computed while they work on step s
+                if (s + 1 < nsteps) {
+                    ok = mbar_wait_spin(x_read, s & 1, abort_flag) && issue_x(s + 1);
+                    if (!ok) break;
+                }
                 // acc1 += P S_b (dV += P^T dO), acc2 += G S_a (dK += dS^T Q, or
-                // dQ += dS K), 64 streamed rows per half as each half lands
+                // dQ += dS K), 64 streamed rows per half as each half lands. P and G of
+                // the 32 streamed rows 32q .. 32q + 31 sit in Y's columns 32q .. 32q + 15
+                // and 32q + 16 .. 32q + 31.
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     ok = mbar_wait_spin(&pg_half[h], s & 1, abort_flag);
@@ -250,14 +272,17 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                     for (int kk = h * (BT / 32); kk < (h + 1) * (BT / 32); ++kk) {
                         const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                        const uint32_t pcol = tY + 32 * (kk >> 1) + 8 * (kk & 1);
                         if (DKDV)
-                            mma_ts(tA1, tX + kk * 8, make_sdesc_sw128(sb + kk * 16 * 128, BT * 128, 1024), idesc_acc,
-                                   acc);
-                        mma_ts(tA2, tY + kk * 8, make_sdesc_sw128(sa + kk * 16 * 128, BT * 128, 1024), idesc_acc, acc);
+                            mma_ts(tA1, pcol, make_sdesc_sw128(sb + kk * 16 * 128, BT * 128, 1024), idesc_acc, acc);
+                        mma_ts(tA2, pcol + 16, make_sdesc_sw128(sa + kk * 16 * 128, BT * 128, 1024), idesc_acc, acc);
                     }
                 }
                 if (!ok) break;
                 tc_commit(&st_empty[bu]);
+                // Y(s+1) over the P and G the accumulating MMAs above read: the tensor
+                // pipe's issue order keeps them intact until read
+                if (s + 1 < nsteps) issue_y(s + 1);
             }
             tc_commit(fin);
             mbar_wait(fin, 0, nullptr);
@@ -320,54 +345,55 @@ __global__ void __launch_bounds__(192, 1)
                 break;
             }
             tc_fence_after();
+            // X into registers at once: X's columns are then free for X(s+1)
+            uint32_t xv[128];
+            tmem_ld64(tX, reinterpret_cast<uint32_t(&)[64]>(xv[0]));
+            tmem_ld64(tX + 64, reinterpret_cast<uint32_t(&)[64]>(xv[64]));
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(x_read);
+            // P of the 128 columns, in place
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                const int col = 2 * i;
+                const float2 nl2 = DKDV ? *reinterpret_cast<const float2*>(lsb + col) : make_float2(nl2_row, nl2_row);
+                const float2 a = ffma2(make_float2(__uint_as_float(xv[2 * i]), __uint_as_float(xv[2 * i + 1])), c2, nl2);
+                xv[2 * i] = __float_as_uint(ex2_approx(a.x));
+                xv[2 * i + 1] = __float_as_uint(ex2_approx(a.y));
+            }
+            if (need_mask) {
+#pragma unroll
+                for (int i = 0; i < 128; ++i)
+                    if (i < lo || i >= hi) xv[i] = 0u;
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(y_full, s & 1, abort_flag))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            // G = P (Y - Delta), 32 columns at a time; P and G of columns 32q .. 32q + 31
+            // go back as bf16 pairs over Y's columns 32q .. 32q + 15 and 32q + 16 .. 32q + 31
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                // P of 64 columns from X
-                float pf[64];
-                {
-                    uint32_t xs[64];
-                    tmem_ld64(tX + h * 64, xs);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int col = h * 64 + 2 * i;
-                        const float2 nl2 =
-                            DKDV ? *reinterpret_cast<const float2*>(lsb + col) : make_float2(nl2_row, nl2_row);
-                        const float2 a =
-                            ffma2(make_float2(__uint_as_float(xs[2 * i]), __uint_as_float(xs[2 * i + 1])), c2, nl2);
-                        pf[2 * i] = ex2_approx(a.x);
-                        pf[2 * i + 1] = ex2_approx(a.y);
-                    }
-                }
-                if (need_mask) {
-#pragma unroll
-                    for (int i = 0; i < 64; ++i) {
-                        const int col = h * 64 + i;
-                        if (col < lo || col >= hi) pf[i] = 0.f;
-                    }
-                }
-                if (h == 0 && !__all_sync(0xffffffffu, mbar_wait(y_full, s & 1, abort_flag))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                // G = P (Y - Delta), 32 columns at a time
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    const int q = 2 * h + q2;
                     uint32_t ys[32], pk[16], gk[16];
-                    tmem_ld32(tY + h * 64 + q * 32, ys);
+                    tmem_ld32(tY + 32 * q, ys);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const int j = q * 32 + 2 * i;  // column inside the half
-                        const float2 ndl = DKDV ? *reinterpret_cast<const float2*>(lsb + BT + h * 64 + j)
-                                                : make_float2(ndl_row, ndl_row);
+                        const int j = 32 * q + 2 * i;  // column
+                        const float2 ndl =
+                            DKDV ? *reinterpret_cast<const float2*>(lsb + BT + j) : make_float2(ndl_row, ndl_row);
                         const float2 t =
                             fadd2(make_float2(__uint_as_float(ys[2 * i]), __uint_as_float(ys[2 * i + 1])), ndl);
-                        const float2 g = fmul2(make_float2(pf[j], pf[j + 1]), t);
-                        pk[i] = pack_bf16x2(pf[j], pf[j + 1]);
+                        const float2 pp = make_float2(__uint_as_float(xv[j]), __uint_as_float(xv[j + 1]));
+                        const float2 g = fmul2(pp, t);
+                        pk[i] = pack_bf16x2(pp.x, pp.y);
                         gk[i] = pack_bf16x2(g.x, g.y);
                     }
-                    if (DKDV) tmem_st16(tX + h * 32 + q * 16, pk);
-                    tmem_st16(tY + h * 32 + q * 16, gk);
+                    if (DKDV) tmem_st16(tY + 32 * q, pk);
+                    tmem_st16(tY + 32 * q + 16, gk);
                 }
                 tmem_st_wait();
                 tc_fence_before();
