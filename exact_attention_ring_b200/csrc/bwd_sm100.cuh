@@ -55,7 +55,7 @@ struct BwdCfg {
     static constexpr int BT = 128;                 // rows of a query tile / keys of a key tile
     static constexpr int CHUNKS = D / 64;
     static constexpr int TILE_BYTES = BT * D * 2;  // one 128 x D bf16 tile
-    static constexpr int NUM_THREADS = 192;
+    static constexpr int NUM_THREADS = 320;
     // [fixed A, B tiles][2 buffers x 2 streamed tiles][lse/delta 2 x 2 x 128 floats][barriers]
     static constexpr int SMEM_USED = 1024 + 2 * TILE_BYTES + 4 * TILE_BYTES + 4 * BT * 4 + 16 * 8 + 16;
     // A block allocates all 512 TMEM columns, so two blocks must never share an
@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdParams p, long 
 // sequence) skip the mask.
 // TMEM: X [0, 128), Y [128, 256), acc1 [256, 256 + D), acc2 [256 + D, 256 + 2D).
 template <int D, bool CAUSAL, bool DKDV>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_fa, const __grid_constant__ CUtensorMap tm_fb,
                     const __grid_constant__ CUtensorMap tm_sa, const __grid_constant__ CUtensorMap tm_sb,
                     const BwdParams p) {
@@ -120,11 +120,11 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* st_empty = bars + 3;   // [2] streamed tiles of a buffer read by every MMA
     uint64_t* x_full = bars + 5;     // X complete
     uint64_t* y_full = bars + 6;     // Y complete
-    uint64_t* pg_half = bars + 7;    // [2] P and G of a half written (4 warp arrivals)
+    uint64_t* pg_half = bars + 7;    // [2] P and G of a half written (its 4 warps)
     uint64_t* l_ready = bars + 9;    // [2] lse/Delta of a buffer staged (4 warp arrivals)
-    uint64_t* l_free = bars + 11;    // [2] lse/Delta of a buffer read (4 warp arrivals)
+    uint64_t* l_free = bars + 11;    // [2] lse/Delta of a buffer read (8 warp arrivals)
     uint64_t* fin = bars + 13;       // every MMA done
-    uint64_t* x_read = bars + 14;    // X in the element-wise warps' registers (4 warp arrivals)
+    uint64_t* x_read = bars + 14;    // X in the element-wise warps' registers (8 warp arrivals)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 15);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -151,16 +151,16 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&st_empty[i], 1);
             mbar_init(&pg_half[i], 4);
             mbar_init(&l_ready[i], 4);
-            mbar_init(&l_free[i], 4);
+            mbar_init(&l_free[i], 8);
         }
         mbar_init(x_full, 1);
         mbar_init(y_full, 1);
         mbar_init(fin, 1);
-        mbar_init(x_read, 4);
+        mbar_init(x_read, 8);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 4) {
+    if (warp == 8) {
         tmem_alloc(tmem_holder, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(192, 1)
         }
     };
 
-    if (warp == 5) {
+    if (warp == 9) {
         // ------------------------------------------------------ producer ----
         if (lane == 0 && nsteps > 0) {
             constexpr uint32_t BOX = BT * 128;
@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(192, 1)
             mbar_wait(fix_full, 0, nullptr);
             for (int i = max(0, s - 2); i < s; ++i) mbar_wait(&st_full[i & 1], (i >> 1) & 1, nullptr);
         }
-    } else if (warp == 4) {
+    } else if (warp == 8) {
         // ---------------------------------------------------- MMA issuer ----
         if (lane == 0 && nsteps > 0) {
             constexpr uint32_t idesc_xy = make_idesc(BT, BT, 0, 0, ElemBf16::fmt);  // A, B K-major
@@ -290,8 +290,11 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------- element-wise -----
-        const int row = warp * 32 + lane;  // TMEM lane: key (dK/dV) or query row (dQ)
-        const uint32_t lb = tmem + (uint32_t(warp * 32) << 16);
+        // warps w and w + 4 share TMEM lane quarter w: w < 4 takes columns
+        // 0 .. 63 (half 0), w >= 4 columns 64 .. 127 (half 1) of the same rows
+        const int quad = warp & 3, grp = warp >> 2;
+        const int row = quad * 32 + lane;  // TMEM lane: key (dK/dV) or query row (dQ)
+        const uint32_t lb = tmem + (uint32_t(quad * 32) << 16);
         const uint32_t tX = lb, tY = lb + 128, tA1 = lb + 256, tA2 = lb + 256 + D;
         const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
         const float LOG2E = 1.4426950408889634f;
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(192, 1)
             ndl_row = -p.delta[r];
         }
         // dK/dV: -lse log2e and -Delta of the streamed query rows, staged in
-        // shared memory one step ahead (each thread one row)
+        // shared memory one step ahead by warps 0-3 (each thread one row)
         auto stage_load = [&](int s, float* nl2, float* ndl) {
             int plane, trow;
             step_src(s, &plane, &trow);
@@ -320,16 +323,18 @@ __global__ void __launch_bounds__(192, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&l_ready[s & 1]);
         };
+        const bool stager = DKDV && grp == 0;
         bool ok = nsteps > 0;
         float pre_nl2 = 0.f, pre_ndl = 0.f;
-        if (DKDV && ok) {
+        if (stager && ok) {
             stage_load(0, &pre_nl2, &pre_ndl);
             stage_store(0, pre_nl2, pre_ndl);
         }
+        const int c0 = 64 * grp;  // this warp's first column
         for (int s = 0; ok && s < nsteps; ++s) {
             int plane, trow;
             step_src(s, &plane, &trow);
-            if (DKDV && s + 1 < nsteps) stage_load(s + 1, &pre_nl2, &pre_ndl);
+            if (stager && s + 1 < nsteps) stage_load(s + 1, &pre_nl2, &pre_ndl);
             const float* lsb = sL + (s & 1) * 2 * BT;
             if (DKDV && !__all_sync(0xffffffffu, mbar_wait(&l_ready[s & 1], (s >> 1) & 1, abort_flag))) {
                 ok = false;
@@ -345,17 +350,16 @@ __global__ void __launch_bounds__(192, 1)
                 break;
             }
             tc_fence_after();
-            // X into registers at once: X's columns are then free for X(s+1)
-            uint32_t xv[128];
-            tmem_ld64(tX, reinterpret_cast<uint32_t(&)[64]>(xv[0]));
-            tmem_ld64(tX + 64, reinterpret_cast<uint32_t(&)[64]>(xv[64]));
+            // this warp's half of X into registers: X's columns are then free for X(s+1)
+            uint32_t xv[64];
+            tmem_ld64(tX + c0, xv);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(x_read);
-            // P of the 128 columns, in place
+            // P of the 64 columns, in place
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const int col = 2 * i;
+            for (int i = 0; i < 32; ++i) {
+                const int col = c0 + 2 * i;
                 const float2 nl2 = DKDV ? *reinterpret_cast<const float2*>(lsb + col) : make_float2(nl2_row, nl2_row);
                 const float2 a = ffma2(make_float2(__uint_as_float(xv[2 * i]), __uint_as_float(xv[2 * i + 1])), c2, nl2);
                 xv[2 * i] = __float_as_uint(ex2_approx(a.x));
@@ -363,8 +367,8 @@ __global__ void __launch_bounds__(192, 1)
             }
             if (need_mask) {
 #pragma unroll
-                for (int i = 0; i < 128; ++i)
-                    if (i < lo || i >= hi) xv[i] = 0u;
+                for (int i = 0; i < 64; ++i)
+                    if (c0 + i < lo || c0 + i >= hi) xv[i] = 0u;
             }
             if (!__all_sync(0xffffffffu, mbar_wait(y_full, s & 1, abort_flag))) {
                 ok = false;
@@ -374,38 +378,33 @@ __global__ void __launch_bounds__(192, 1)
             // G = P (Y - Delta), 32 columns at a time; P and G of columns 32q .. 32q + 31
             // go back as bf16 pairs over Y's columns 32q .. 32q + 15 and 32q + 16 .. 32q + 31
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int q2 = 0; q2 < 2; ++q2) {
+                const int q = 2 * grp + q2;
+                uint32_t ys[32], pk[16], gk[16];
+                tmem_ld32(tY + 32 * q, ys);
 #pragma unroll
-                for (int q2 = 0; q2 < 2; ++q2) {
-                    const int q = 2 * h + q2;
-                    uint32_t ys[32], pk[16], gk[16];
-                    tmem_ld32(tY + 32 * q, ys);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int j = 32 * q + 2 * i;  // column
-                        const float2 ndl =
-                            DKDV ? *reinterpret_cast<const float2*>(lsb + BT + j) : make_float2(ndl_row, ndl_row);
-                        const float2 t =
-                            fadd2(make_float2(__uint_as_float(ys[2 * i]), __uint_as_float(ys[2 * i + 1])), ndl);
-                        const float2 pp = make_float2(__uint_as_float(xv[j]), __uint_as_float(xv[j + 1]));
-                        const float2 g = fmul2(pp, t);
-                        pk[i] = pack_bf16x2(pp.x, pp.y);
-                        gk[i] = pack_bf16x2(g.x, g.y);
-                    }
-                    if (DKDV) tmem_st16(tY + 32 * q, pk);
-                    tmem_st16(tY + 32 * q + 16, gk);
+                for (int i = 0; i < 16; ++i) {
+                    const int j = 32 * q2 + 2 * i;  // column inside this warp's half
+                    const float2 ndl = DKDV ? *reinterpret_cast<const float2*>(lsb + BT + c0 + j)
+                                            : make_float2(ndl_row, ndl_row);
+                    const float2 t = fadd2(make_float2(__uint_as_float(ys[2 * i]), __uint_as_float(ys[2 * i + 1])), ndl);
+                    const float2 pp = make_float2(__uint_as_float(xv[j]), __uint_as_float(xv[j + 1]));
+                    const float2 g = fmul2(pp, t);
+                    pk[i] = pack_bf16x2(pp.x, pp.y);
+                    gk[i] = pack_bf16x2(g.x, g.y);
                 }
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&pg_half[h]);
+                if (DKDV) tmem_st16(tY + 32 * q, pk);
+                tmem_st16(tY + 32 * q + 16, gk);
             }
-            if (!ok) break;
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pg_half[grp]);
             if (DKDV) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&l_free[s & 1]);
-                if (s + 1 < nsteps) {
-                    // buffer (s + 1) & 1 was last read in step s - 1
+                if (stager && s + 1 < nsteps) {
+                    // buffer (s + 1) & 1 was last read in step s - 1 (by both halves)
                     if (s >= 1 &&
                         !__all_sync(0xffffffffu, mbar_wait(&l_free[(s + 1) & 1], ((s - 1) >> 1) & 1, abort_flag))) {
                         ok = false;
@@ -422,13 +421,15 @@ __global__ void __launch_bounds__(192, 1)
             const bool in_seq = fixed_pos < p.N;
             const size_t out_row =
                 static_cast<size_t>(DKDV ? b * p.Hkv + hfix : b * p.Hq + hfix) * p.N + (in_seq ? fixed_pos : 0);
-#pragma unroll
-            for (int which = 0; which < (DKDV ? 2 : 1); ++which) {
+            // dK/dV: warps 0-3 write dV, warps 4-7 dK; dQ: each group half of the columns
+            {
+                const int which = DKDV ? grp : 1;
                 __nv_bfloat16* dst = (DKDV ? (which == 0 ? p.dv : p.dk) : p.dq) + out_row * D;
-                const uint32_t src = DKDV ? (which == 0 ? tA1 : tA2) : tA2;
-                const float f = (DKDV && which == 0) ? 1.f : p.scale;  // dK, dQ carry the scale
+                const uint32_t src = which == 0 ? tA1 : tA2;
+                const float f = which == 0 ? 1.f : p.scale;  // dK, dQ carry the scale
+                const int c_lo = DKDV ? 0 : grp * (D / 64), c_hi = DKDV ? D / 32 : (grp + 1) * (D / 64);
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = c_lo; c < c_hi; ++c) {
                     uint32_t r3[32];
                     tmem_ld32(src + c * 32, r3);
                     if (in_seq) {
