@@ -109,8 +109,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kCombineMaxSplits = 12000;
 
 template <int D, bool CAUSAL, bool F32OUT, class E>
-attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
-                         cudaStream_t stream) {
+attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                         const FwdParams& p, cudaStream_t stream) {
     using C = FwdCfg<D>;
     auto kern = attn_fwd_kernel<D, CAUSAL, F32OUT, E>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
@@ -121,7 +121,7 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
         return ATTN_ERR_CUDA;
     const int grid = p.n_items < sms ? p.n_items : sms;
-    if (launch_pdl(kern, dim3(grid), dim3(C::NUM_THREADS), C::SMEM_BYTES, stream, tq, tk, tv, p) != cudaSuccess)
+    if (launch_pdl(kern, dim3(grid), dim3(C::NUM_THREADS), C::SMEM_BYTES, stream, tq, tk, tv, to, p) != cudaSuccess)
         return ATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -172,10 +172,14 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
         return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (static_cast<long long>(B) * Hq > 65535LL * 1024) return ATTN_ERR_INVALID_ARG;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!make_map<E>(&tq, q, d, N, B * Hq, 128) || !make_map<E>(&tk, k, d, N, B * Hkv, 128) ||
         !make_map<E>(&tv, v, d, N, B * Hkv, 128))
         return ATTN_ERR_CUDA;
+    // O as 32-row boxes for the epilogue's bulk stores (16-bit outputs; the fp32
+    // output is written by the threads and does not use it)
+    if (F32OUT) to = tq;
+    else if (!make_map<E>(&to, o, d, N, B * Hq, 32)) return ATTN_ERR_CUDA;
     FwdParams p;
     p.o = o;
     p.lse = lse;
@@ -191,9 +195,10 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
     p.sched_slot = static_cast<int>(launch_seq.fetch_add(1u) % kFwdSchedSlots);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d == 128)
-        return causal ? launch_fwd<128, true, F32OUT, E>(tq, tk, tv, p, st)
-                      : launch_fwd<128, false, F32OUT, E>(tq, tk, tv, p, st);
-    return causal ? launch_fwd<64, true, F32OUT, E>(tq, tk, tv, p, st) : launch_fwd<64, false, F32OUT, E>(tq, tk, tv, p, st);
+        return causal ? launch_fwd<128, true, F32OUT, E>(tq, tk, tv, to, p, st)
+                      : launch_fwd<128, false, F32OUT, E>(tq, tk, tv, to, p, st);
+    return causal ? launch_fwd<64, true, F32OUT, E>(tq, tk, tv, to, p, st)
+                  : launch_fwd<64, false, F32OUT, E>(tq, tk, tv, to, p, st);
 }
 
 template <int D, bool CAUSAL, bool DKDV>

@@ -160,7 +160,8 @@ __device__ __forceinline__ float max64(const float (&v)[64]) {
 template <int D, bool CAUSAL, bool F32OUT, class E>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                    const FwdParams p) {
     using C = FwdCfg<D>;
     constexpr int BM = C::BM, BN = C::BN, SLOTS = C::SLOTS;
     extern __shared__ uint8_t smem_raw[];
@@ -586,11 +587,14 @@ __global__ void __launch_bounds__(384, 1)
                     __syncwarp();
                 }
             } else {
-            auto* ob = static_cast<typename E::T*>(p.o);
 #pragma unroll
             for (int half = 0; half < D / 64; ++half) {
+                // the staging buffer is free once the bulk store that read it last is done
+                if (lane == 0) bulk_wait_read_all();
+                __syncwarp();
                 // this lane's row, columns [64*half, 64*half + 64): 128 bytes as 8
-                // chunks of 16; chunk i of row r sits at slot i ^ (r & 7)
+                // chunks of 16; chunk i of row r sits at slot i ^ (r & 7), the layout
+                // of a 128-byte-swizzled 32-row box of O
 #pragma unroll
                 for (int c2 = 0; c2 < 2; ++c2) {
                     const int c = half * 2 + c2;
@@ -613,22 +617,21 @@ __global__ void __launch_bounds__(384, 1)
                         *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = v4;
                     }
                 }
+                // one bulk tensor store of the warp's 32 rows x 64 columns (rows past N
+                // are clipped by the tensor map); the warp goes on at once
+                fence_proxy_async_smem();
                 __syncwarp();
-                // read back: lane = 8 * (row within a group of 4) + chunk, 4 rows per store
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int rr = 4 * k + (lane >> 3), chunk = lane & 7;
-                    const uint4 v4 = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((chunk ^ (rr & 7)) << 4));
-                    if (row0 + rr < p.N)
-                        *reinterpret_cast<uint4*>(ob + (static_cast<size_t>(item.bh) * p.N + row0 + rr) * D +
-                                                  half * 64 + chunk * 8) = v4;
+                if (lane == 0) {
+                    tma_store_3d(&tm_o, stage, half * 64, row0, item.bh);
+                    bulk_commit();
                 }
-                __syncwarp();
             }
             }
             if (grow < p.N)
                 p.lse[static_cast<size_t>(item.bh) * p.N + grow] = (m_used + log2f(l)) * 0.69314718055994530942f;
         }
+        // the bulk stores read the staging buffers: complete before the CTA exits
+        if (!F32OUT && lane == 0) bulk_wait_all();
     }
 
     tc_fence_before();
