@@ -30,6 +30,16 @@
  *    are then undefined); attn_device_status() reads and clears that word.
  *  - LSE is the natural-log log-sum-exp of the scaled, masked scores of a row:
  *    lse_i = ln sum_{j visible} exp(scale * q_i . k_j).
+ *  - Kernels are launched with programmatic stream serialization: a kernel's
+ *    blocks may be scheduled while the previous kernel in the stream finishes,
+ *    but each waits for that kernel's completion before its first access to
+ *    device memory, so the stream's order of memory effects is unchanged.
+ *  - Calls may be captured in CUDA graphs. A non-causal attn_fwd (and
+ *    attn_fwd_f16, attn_fwd_f32) hands out its work items through one of 64
+ *    device counters, taken by successive calls in turn and back at zero when
+ *    the call's kernel ends: at most 64 such calls may be in flight at once,
+ *    and a captured call keeps its counter at every replay, so replays of one
+ *    graph must not run concurrently with each other.
  */
 #ifndef EXACT_ATTENTION_RING_B200_ATTN_H
 #define EXACT_ATTENTION_RING_B200_ATTN_H
