@@ -74,8 +74,8 @@ NCU_TRAFFIC = {
     "decode": {"bytes_per_launch": 536959744 + 3461376, "source_sha": "eaaf414296e5590d"},
     "decode_b1_l32k": {"bytes_per_launch": 134302976 + 3129856, "source_sha": "eaaf414296e5590d"},
     "decode_b8_l32k": {"bytes_per_launch": 1073927168 + 3971072, "source_sha": "eaaf414296e5590d"},
-    "attn_fwd_causal": {"bytes_per_launch": 137771008 + 13184000, "source_sha": "4a7ee4f42a05d865"},
-    "attn_fwd_noncausal": {"bytes_per_launch": 100734464 + 13857536, "source_sha": "4a7ee4f42a05d865"},
+    "attn_fwd_causal": {"bytes_per_launch": 131980800 + 12869120, "source_sha": "7eb65e92f430f85e"},
+    "attn_fwd_noncausal": {"bytes_per_launch": 100789760 + 13249536, "source_sha": "7eb65e92f430f85e"},
 }
 
 

@@ -20,10 +20,11 @@
 // CTAs finish together. 384 threads,
 // warp-specialised:
 //   warps 0-3   softmax of query tile 0, one thread per row (TMEM lane), and
-//               its epilogue: O/l rounded to the input type (or kept in fp32
-//               for the F32OUT kernels), staged per warp in shared memory
-//               (16-byte chunks XOR-swizzled) and read back so that every
-//               store writes whole 128-byte row segments;
+//               its epilogue: O/l rounded to the input type, staged per warp in
+//               shared memory as a 128-byte-swizzled 32-row box and written by
+//               one bulk tensor store per 64 columns (the F32OUT kernels keep O
+//               in fp32, read the staging back and store whole 128-byte row
+//               segments);
 //   warps 4-7   the same for query tile 1;
 //   warp 8, 9   MMA issuers, one per query tile. A thread that has just issued
 //               tcgen05.mma cannot act on an mbarrier for several hundred cycles,
@@ -31,7 +32,9 @@
 //   warps 10,11 TMA producers: the Q tiles of each item, then K_j and V_j into a
 //               ring of shared-memory slots (full/empty mbarriers). One issuing
 //               thread streams TMA boxes one after another, so the boxes of
-//               every tile are split between two threads.
+//               every tile are split between two threads. They run key tiles
+//               ahead and wait with suspended try_wait, taking no issue slots
+//               from the softmax warps of their sub-partitions.
 // Per query tile t and key tile j:
 //   S_t = Q_t K_j^T           tcgen05.mma (A, B K-major in smem) -> TMEM S_t;
 //   softmax                   pass 1 reads S_t and takes the row max; when it has
