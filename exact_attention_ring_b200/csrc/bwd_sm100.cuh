@@ -22,8 +22,9 @@
 //   bwd_tile_kernel, !DKDV  one 128-row query tile of one (batch, query head)
 //                           per block: S = Q K^T and dP = dO V^T per key tile,
 //                           dS (bf16) over dP, dQ += dS K (then times scale).
-// 192 threads each: warps 0-3 element-wise work and epilogue (thread = TMEM
-// lane), warp 4 the MMA issuer, warp 5 the TMA producer. Within a step the
+// 320 threads each: warps 0-7 element-wise work and epilogue (thread = TMEM
+// lane; warps w and w + 4 share lane quarter w and split its 128 columns in
+// halves), warp 8 the MMA issuer, warp 9 the TMA producer. Within a step the
 // element-wise pass reads S^T into registers at once, so the next step's S^T
 // MMAs run while it computes P (as dP^T is completing) and dS; P and dS go
 // back as bf16 over dP^T's columns, a quarter at a time, and are handed over
