@@ -399,8 +399,8 @@ attn_status_t attn_quant_fp8(const void* x, void* codes, float* scales, int plan
     const dim3 grid(nblk, planes);
     if (!per_plane && !transpose) {
         // per-block scales, row-major codes: one pass over x
-        if (d == 128) launch_pdl(fp8_quant_rows_kernel<128, false>, grid, dim3(256), 0, st, p);
-        else launch_pdl(fp8_quant_rows_kernel<64, false>, grid, dim3(256), 0, st, p);
+        if (d == 128) launch_pdl(fp8_quant_rows_kernel<128, false>, grid, dim3(kQuantRowsThreads), 0, st, p);
+        else launch_pdl(fp8_quant_rows_kernel<64, false>, grid, dim3(kQuantRowsThreads), 0, st, p);
         return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
     }
     if (d == 128) {
@@ -431,8 +431,8 @@ attn_status_t attn_quant_fp8_rotate(const void* x, const float* signs, void* cod
     p.rot_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const dim3 grid(nblk, planes);
-    if (d == 128) launch_pdl(fp8_quant_rows_kernel<128, true>, grid, dim3(256), 0, st, p);
-    else launch_pdl(fp8_quant_rows_kernel<64, true>, grid, dim3(256), 0, st, p);
+    if (d == 128) launch_pdl(fp8_quant_rows_kernel<128, true>, grid, dim3(kQuantRowsThreads), 0, st, p);
+    else launch_pdl(fp8_quant_rows_kernel<64, true>, grid, dim3(kQuantRowsThreads), 0, st, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

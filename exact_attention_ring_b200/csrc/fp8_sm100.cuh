@@ -67,7 +67,8 @@ struct QuantParams {
 };
 
 // One pass over one 128-row block of a plane, for the per-block, row-major codes
-// of Q and K: each warp holds 16 rows in registers (lane l has elements
+// of Q and K (512 threads, so that an SM holds enough blocks' loads in flight):
+// each of the 16 warps holds 8 rows in registers (lane l has elements
 // l*E .. l*E+E-1, E = D/32), optionally applies the rotation of incoherent
 // processing (FlashAttention-3 page, FP8 paragraph; reading: y = H (sigma o x) /
 // sqrt(D), H the Sylvester Hadamard matrix, sigma random signs shared by Q and
@@ -76,11 +77,12 @@ struct QuantParams {
 // of span 1, 2, ..., D/2 in that order (spans below E inside a lane, the rest
 // across lanes by shuffles) and one multiplication by rot_scale: every element
 // takes exactly the fp32 operations of the transform's definition, in its order.
+constexpr int kQuantRowsThreads = 512;
 template <int D, bool ROTATE>
-__global__ void __launch_bounds__(256) fp8_quant_rows_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(kQuantRowsThreads) fp8_quant_rows_kernel(const QuantParams p) {
     grid_dep_wait();  // the previous kernel's writes are visible from here on
     grid_dep_launch();
-    constexpr int E = D / 32, RPW = 16;
+    constexpr int NW = kQuantRowsThreads / 32, E = D / 32, RPW = 128 / NW;
     const int blk = blockIdx.x, plane = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r0 = blk * 128, rows = min(128, p.N - r0);
@@ -144,12 +146,12 @@ __global__ void __launch_bounds__(256) fp8_quant_rows_kernel(const QuantParams p
         for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(v[i][e]));  // rows past N hold zeros
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    __shared__ float wm[8];
+    __shared__ float wm[NW];
     if (lane == 0) wm[warp] = m;
     __syncthreads();
     float amax = wm[0];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) amax = fmaxf(amax, wm[w]);
+    for (int w = 1; w < NW; ++w) amax = fmaxf(amax, wm[w]);
     const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
     if (threadIdx.x == 0) p.scales[static_cast<size_t>(plane) * p.nblk + blk] = sc;
     uint8_t* dst = p.codes + (static_cast<size_t>(plane) * p.N + r0) * D;
