@@ -230,37 +230,47 @@ __global__ void __launch_bounds__(256) fp8_quant_kernel(const QuantParams p) {
                 make_uint2(uint32_t(c[0]) | (uint32_t(c[1]) << 16), uint32_t(c[2]) | (uint32_t(c[3]) << 16));
         }
     } else {
-        // codes of the block's 128 rows (zero past N), then written out as D rows
-        // of 128 keys each
-        __shared__ uint8_t tile[128][D + 16];
-        for (int i = threadIdx.x; i < 128 * D / 8; i += 256) {
-            const int r = i / (D / 8), c8 = (i % (D / 8)) * 8;
-            uint16_t c[4] = {0, 0, 0, 0};
-            if (r < rows) {
-                const uint4 u = *reinterpret_cast<const uint4*>(src + static_cast<size_t>(r) * D + c8);
-                const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+        // codes of the block's 128 rows (zero past N), transposed through shared
+        // memory and written out as D rows of 128 keys each. Lane l converts keys
+        // 4l .. 4l + 3 at 8 dimensions and stores, per dimension, the four codes
+        // as one word (key-consecutive words: no bank conflicts); the rows of the
+        // tile are 33 words apart, so the read-back of 16 keys of a dimension per
+        // thread is conflict-free as well.
+        __shared__ uint32_t tileT[D][33];
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        const int kq = lane;  // keys 4kq .. 4kq + 3
+        for (int g = warp; g < D / 8; g += 8) {
+            const int c8 = g * 8;
+            uint16_t c[4][4];  // [key][dimension pair]
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(h[e]);
-                    c[e] = e4m3x2(__fdiv_rn(f.x, s), __fdiv_rn(f.y, s));
+            for (int j = 0; j < 4; ++j) {
+                const int r = 4 * kq + j;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) c[j][e] = 0;
+                if (r < rows) {
+                    const uint4 u = *reinterpret_cast<const uint4*>(src + static_cast<size_t>(r) * D + c8);
+                    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(h[e]);
+                        c[j][e] = e4m3x2(__fdiv_rn(f.x, s), __fdiv_rn(f.y, s));
+                    }
                 }
             }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                tile[r][c8 + 2 * e] = uint8_t(c[e] & 0xff);
-                tile[r][c8 + 2 * e + 1] = uint8_t(c[e] >> 8);
+            for (int e = 0; e < 8; ++e) {
+                const int sh = (e & 1) * 8;
+                tileT[c8 + e][kq] = uint32_t((c[0][e >> 1] >> sh) & 0xff) | (uint32_t((c[1][e >> 1] >> sh) & 0xff) << 8) |
+                                    (uint32_t((c[2][e >> 1] >> sh) & 0xff) << 16) |
+                                    (uint32_t((c[3][e >> 1] >> sh) & 0xff) << 24);
             }
         }
         __syncthreads();
         uint8_t* dst = p.codes + static_cast<size_t>(plane) * D * p.Np + r0;
         for (int i = threadIdx.x; i < D * 8; i += 256) {
-            const int t = i >> 3, k0 = (i & 7) * 16;  // dimension t, keys [k0, k0 + 16)
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                w[e] = uint32_t(tile[k0 + 4 * e][t]) | (uint32_t(tile[k0 + 4 * e + 1][t]) << 8) |
-                       (uint32_t(tile[k0 + 4 * e + 2][t]) << 16) | (uint32_t(tile[k0 + 4 * e + 3][t]) << 24);
-            *reinterpret_cast<uint4*>(dst + static_cast<size_t>(t) * p.Np + k0) = make_uint4(w[0], w[1], w[2], w[3]);
+            const int t = i >> 3, q = i & 7;  // dimension t, keys [16q, 16q + 16)
+            *reinterpret_cast<uint4*>(dst + static_cast<size_t>(t) * p.Np + 16 * q) =
+                make_uint4(tileT[t][4 * q], tileT[t][4 * q + 1], tileT[t][4 * q + 2], tileT[t][4 * q + 3]);
         }
     }
 }
