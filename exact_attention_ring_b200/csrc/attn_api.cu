@@ -108,22 +108,58 @@ constexpr float kLog2e = 1.4426950408889634f;
 // static words it must stay under the 48 KiB a launch gets without opting in.
 constexpr int kCombineMaxSplits = 12000;
 
-template <int D, bool CAUSAL, bool F32OUT, class E>
-attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
-                         const FwdParams& p, cudaStream_t stream) {
+template <int D, bool CAUSAL, bool F32OUT, class E, bool SPLIT>
+attn_status_t launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const CUtensorMap& to, const FwdParams& p, int grid, cudaStream_t stream) {
     using C = FwdCfg<D>;
-    auto kern = attn_fwd_kernel<D, CAUSAL, F32OUT, E>;
+    auto kern = attn_fwd_kernel<D, CAUSAL, F32OUT, E, SPLIT>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
+    if (launch_pdl(kern, dim3(grid), dim3(C::NUM_THREADS), C::SMEM_BYTES, stream, tq, tk, tv, to, p) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Non-causal launches count their work items in a device counter slot; successive
+// launches take successive slots (shared by every element type and output kind).
+std::atomic<unsigned int> g_fwd_launch_seq{0};
+int next_fwd_slot() { return static_cast<int>(g_fwd_launch_seq.fetch_add(1u) % kFwdSchedSlots); }
+
+template <int D, bool CAUSAL, bool F32OUT, class E>
+attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                         const FwdParams& p0, cudaStream_t stream) {
     // persistent grid: one CTA per SM, each walking its share of the work items
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
         return ATTN_ERR_CUDA;
-    const int grid = p.n_items < sms ? p.n_items : sms;
-    if (launch_pdl(kern, dim3(grid), dim3(C::NUM_THREADS), C::SMEM_BYTES, stream, tq, tk, tv, to, p) != cudaSuccess)
-        return ATTN_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    FwdParams p = p0;
+    p.block0 = 0;
+    if constexpr (!CAUSAL) {
+        // Non-causal items all cost the same, so a last round of r <= SMs/2 query
+        // blocks would leave most CTAs idle for a whole item. Those blocks go to a
+        // second launch, right behind the first (programmatic dependent launch),
+        // as two 128-row items each: both query tiles of a CTA on the same rows,
+        // half of the key tiles each, merged at the end, so the last round takes
+        // about half as long. Needs at least two key tiles.
+        const int rem = p.n_items % sms;
+        if ((p.N + 127) / 128 >= 2 && rem > 0 && 2 * rem <= sms) {
+            const int n_full = p.n_items - rem;
+            if (n_full > 0) {
+                p.n_items = n_full;
+                p.sched_slot = next_fwd_slot();
+                const attn_status_t st = launch_fwd_kernel<D, CAUSAL, F32OUT, E, false>(tq, tk, tv, to, p, sms, stream);
+                if (st != ATTN_OK) return st;
+            }
+            p.block0 = n_full;
+            p.n_items = 2 * rem;
+            p.sched_slot = next_fwd_slot();
+            return launch_fwd_kernel<D, CAUSAL, F32OUT, E, true>(tq, tk, tv, to, p, p.n_items, stream);
+        }
+        p.sched_slot = next_fwd_slot();
+    }
+    return launch_fwd_kernel<D, CAUSAL, F32OUT, E, false>(tq, tk, tv, to, p, p.n_items < sms ? p.n_items : sms,
+                                                          stream);
 }
 
 template <int D, class E>
@@ -189,10 +225,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
     if (items > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
     p.n_items = static_cast<int>(items);
     p.scale_log2 = scale * kLog2e;
-    // each non-causal launch counts its work items in its own slot; launches that
-    // use one slot at the same time (kFwdSchedSlots launches in flight) would share it
-    static std::atomic<unsigned int> launch_seq{0};
-    p.sched_slot = static_cast<int>(launch_seq.fetch_add(1u) % kFwdSchedSlots);
+    p.sched_slot = 0;  // taken by launch_fwd for non-causal launches
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d == 128)
         return causal ? launch_fwd<128, true, F32OUT, E>(tq, tk, tv, to, p, st)

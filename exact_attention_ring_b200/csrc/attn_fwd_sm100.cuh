@@ -17,7 +17,12 @@
 // K/V tiles through L2, and a CTA takes its first item by its index and each
 // later one from a per-launch counter (the first producer thread takes it and
 // hands it to the other roles through a small ring in shared memory), so the
-// CTAs finish together. 384 threads,
+// CTAs finish together. A non-causal problem whose last round would hold at most
+// half as many query blocks as there are SMs runs that round as a second launch
+// (the SPLIT kernel) in 128-row halves: the two query tiles of a CTA take the same
+// rows against the first and the second half of the key tiles (each K/V tile
+// then serves one tile only), and tile 1 merges the two partial results as the
+// online softmax merges two blocks of keys. 384 threads,
 // warp-specialised:
 //   warps 0-3   softmax of query tile 0, one thread per row (TMEM lane), and
 //               its epilogue: O/l rounded to the input type, staged per warp in
@@ -67,7 +72,8 @@ struct FwdParams {
     float* lse;        // [B, Hq, N]
     int B, Hq, Hkv, N;
     int n_qblocks;     // ceil(N / 256)
-    int n_items;       // n_qblocks * B * Hq
+    int n_items;       // work items of this launch
+    int block0;        // split launches: the first query block; item w is half w & 1 of block block0 + w / 2
     float scale_log2;  // scale * log2(e)
     int sched_slot;    // this launch's work counter in g_fwd_sched
 };
@@ -97,8 +103,8 @@ struct FwdCfg {
     static constexpr int NUM_PRODUCERS = 2;
     static constexpr int ITEM_RING = 4;  // work items handed from the fetching thread to the other roles
     // q_full, q_empty, slot_full, slot_empty, s_full, p_full, o_done, o_free, turn, drain, p_half,
-    // item_full, item_empty
-    static constexpr int NUM_BARRIERS = 2 * 2 + 2 * SLOTS + 7 * 2 + 2 * ITEM_RING;
+    // item_full, item_empty, merge
+    static constexpr int NUM_BARRIERS = 2 * 2 + 2 * SLOTS + 7 * 2 + 2 * ITEM_RING + 1;
     // item readers: the second producer, the two MMA issuers and the eight softmax warps
     static constexpr int ITEM_READERS = 11;
     static constexpr int SMEM_BYTES = 1024 + TILES * Q_TILE_BYTES + SLOTS * TILE_BYTES + 8 * STAGE_O_BYTES +
@@ -115,15 +121,28 @@ __device__ __forceinline__ int fwd_work_index(int r) {
     return r * G + ((r & 1) ? (G - 1 - c) : c);
 }
 
-// One work item: a 256-row query block of one (batch, head).
+// One work item: a 256-row query block of one (batch, head), query tile t taking
+// rows row0[t] .. row0[t] + 127 against key tiles 0 .. nk_t - 1. The items of a
+// split launch (the SPLIT kernels, used for the last round of a non-causal
+// problem) are 128-row halves of blocks: both query tiles take the same rows,
+// tile 0 against key tiles [0, nk0) and tile 1 against [kb1, kb1 + nk1), and the
+// two partial results are merged in the epilogue.
 struct FwdItem {
     int qb, bh, b, h, hk;
-    int nk0, nk1;  // key tiles needed by query tile 0 and 1 (nk1 - nk0 is 0 or 1)
+    int nk0, nk1;  // key tiles of query tile 0 and 1 (nk1 - nk0 is 0 or 1)
+    int row0[2];   // first query row of each tile
+    int kb1;       // first key tile of tile 1 (0 unless split)
+    bool split;
 };
 
-template <bool CAUSAL>
+template <bool CAUSAL, bool SPLIT>
 __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int w) {
     FwdItem it;
+    int half = 0;  // split items: which 128-row half of the block
+    if (SPLIT) {
+        half = w & 1;
+        w = p.block0 + (w >> 1);
+    }
     if (CAUSAL) {
         // heaviest blocks first: every (batch, head) at the last query block, then
         // at the one before, ...
@@ -140,11 +159,66 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int w) {
     it.h = it.bh % p.Hq;
     it.hk = it.h / (p.Hq / p.Hkv);
     const int n_kv = (p.N + 127) / 128;
-    it.nk0 = CAUSAL ? min(2 * it.qb + 1, n_kv) : n_kv;
-    it.nk1 = CAUSAL ? min(2 * it.qb + 2, n_kv) : n_kv;
+    it.split = SPLIT;
+    if (SPLIT) {
+        it.nk0 = n_kv / 2;
+        it.nk1 = n_kv - it.nk0;
+        it.kb1 = it.nk0;
+        it.row0[0] = it.row0[1] = it.qb * 256 + half * 128;
+    } else {
+        it.nk0 = CAUSAL ? min(2 * it.qb + 1, n_kv) : n_kv;
+        it.nk1 = CAUSAL ? min(2 * it.qb + 2, n_kv) : n_kv;
+        it.kb1 = 0;
+        it.row0[0] = it.qb * 256;
+        it.row0[1] = it.qb * 256 + 128;
+    }
     return it;
 }
 
+// K/V loads of an item, in the order the producers issue them. A whole item
+// streams K_0 V_0 K_1 V_1 ... for both tiles. A split item's loads each serve one
+// tile, in the order its two MMA issuers consume them: K_0 of tile 0 and of tile
+// 1, then per key step s the V_s and K_(s+1) of tile 0, then those of tile 1
+// (leaving out what does not exist), so that a slot is never held up behind the
+// other tile's later release.
+__device__ __forceinline__ int fwd_item_loads(const FwdItem& it) { return 2 * (it.split ? it.nk0 + it.nk1 : it.nk1); }
+// Load index (within the item) of K (v = false) or V (v = true) of query tile t's
+// key step j. For a split item with h = nk0: V_t(s) = 2 + 4s + 2t and K_t(s+1)
+// right after it while s + 1 < h; V_0(h-1), V_1(h-1) follow at 4h-2, 4h-1, then
+// tile 1's extra step (nk1 = h + 1) has K_1(h) at 4h and V_1(h) at 4h+1.
+__device__ __forceinline__ int fwd_load_index(const FwdItem& it, int t, int j, bool v) {
+    if (!it.split) return 2 * j + (v ? 1 : 0);
+    const int h = it.nk0;
+    if (v) {
+        if (j < h - 1) return 2 + 4 * j + 2 * t;
+        return j == h - 1 ? 4 * h - 2 + t : 4 * h + 1;
+    }
+    if (j == 0) return t;
+    if (j < h) return 3 + 4 * (j - 1) + 2 * t;
+    return 4 * h;  // K_1(h)
+}
+// Load i of the item: whether it is a V tile, and its key tile.
+__device__ __forceinline__ bool fwd_load_kind(const FwdItem& it, int i, int* key_tile) {
+    if (!it.split) {
+        *key_tile = i >> 1;
+        return (i & 1) != 0;
+    }
+    const int h = it.nk0;
+    int t, step;
+    bool v;
+    if (i < 2) {
+        t = i; step = 0; v = false;
+    } else if (i < 4 * h - 2) {
+        const int s = (i - 2) >> 2, r = (i - 2) & 3;
+        t = r >> 1; v = (r & 1) == 0; step = v ? s : s + 1;
+    } else if (i < 4 * h) {
+        t = i - (4 * h - 2); step = h - 1; v = true;
+    } else {
+        t = 1; step = h; v = i == 4 * h + 1;
+    }
+    *key_tile = step + (t ? it.kb1 : 0);
+    return v;
+}
 
 // Max of 64 values with eight independent chains of 3-input max.
 __device__ __forceinline__ float max64(const float (&v)[64]) {
@@ -160,7 +234,7 @@ __device__ __forceinline__ float max64(const float (&v)[64]) {
     return max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
-template <int D, bool CAUSAL, bool F32OUT, class E>
+template <int D, bool CAUSAL, bool F32OUT, class E, bool SPLIT>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -186,7 +260,8 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* p_half = drain + 2;              // [2] first half of P_t written (4 warp arrivals)
     uint64_t* item_full = p_half + 2;          // [ITEM_RING] work item r published
     uint64_t* item_empty = item_full + C::ITEM_RING;  // [ITEM_RING] read by every role (ITEM_READERS arrivals)
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(item_empty + C::ITEM_RING);
+    uint64_t* merge_bar = item_empty + C::ITEM_RING;  // split item: tile 0's row max and sum published (4 warps)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(merge_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* item_ring = reinterpret_cast<volatile int*>(tmem_holder + 4);  // [ITEM_RING]
 
@@ -212,6 +287,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&item_full[i], 1);
             mbar_init(&item_empty[i], C::ITEM_READERS);
         }
+        if (SPLIT) mbar_init(merge_bar, 4);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -275,7 +351,7 @@ __global__ void __launch_bounds__(384, 1)
                 const int w = CAUSAL ? fwd_work_index(r) : me == 0 ? publish_item(r, next_w) : read_item(r);
                 if (w < 0) { ok = false; break; }
                 if (w >= p.n_items) break;
-                const FwdItem item = fwd_item<CAUSAL>(p, w);
+                const FwdItem item = fwd_item<CAUSAL, SPLIT>(p, w);
                 const int zq = item.b * p.Hq + item.h, zkv = item.b * p.Hkv + item.hk;
                 // issue (this producer's boxes of) K/V load i of the item
                 auto issue_kv = [&](int i) -> bool {
@@ -286,13 +362,15 @@ __global__ void __launch_bounds__(384, 1)
                     if (!mine) return true;
                     const int slot = gi % SLOTS, use = gi / SLOTS;
                     if (use > 0 && !mbar_wait_park(&slot_empty[slot], (use - 1) & 1, abort_flag)) return false;
+                    int kt = i >> 1;
                     const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;
+                    if constexpr (SPLIT) tm = fwd_load_kind(item, i, &kt) ? &tm_v : &tm_k;
                     uint8_t* dst = sKV + slot * C::TILE_BYTES;
 #pragma unroll
                     for (int c = 0; c < C::CHUNKS; ++c) {
                         if ((gi * C::CHUNKS + c) % C::NUM_PRODUCERS != me) continue;
                         mbar_arrive_expect_tx(&slot_full[slot], BOX_BYTES);
-                        tma_load_3d(dst + c * BOX_BYTES, tm, &slot_full[slot], c * 64, (i >> 1) * BN, zkv);
+                        tma_load_3d(dst + c * BOX_BYTES, tm, &slot_full[slot], c * 64, kt * BN, zkv);
                     }
                     return true;
                 };
@@ -308,7 +386,7 @@ __global__ void __launch_bounds__(384, 1)
                         if ((t * C::CHUNKS + c) % C::NUM_PRODUCERS != me) continue;
                         mbar_arrive_expect_tx(&q_full[t], BM * 128);
                         tma_load_3d(sQ + t * C::Q_TILE_BYTES + c * BM * 128, &tm_q, &q_full[t], c * 64,
-                                    item.qb * 2 * BM + t * BM, zq);
+                                    SPLIT ? item.row0[t] : item.qb * 2 * BM + t * BM, zq);
                     }
                     return true;
                 };
@@ -318,10 +396,11 @@ __global__ void __launch_bounds__(384, 1)
                 // causal item), then the rest.
                 // the first producer takes the next item two key tiles before this
                 // item's last loads
-                const int take_at = max(2, 2 * item.nk1 - 4);
+                const int n_loads = SPLIT ? fwd_item_loads(item) : 2 * item.nk1;
+                const int take_at = max(2, n_loads - 4);
                 bool taken = false;
                 ok = issue_q(0) && issue_kv(0) && issue_kv(1) && issue_q(1);
-                for (int i = 2; ok && i < 2 * item.nk1; ++i) {
+                for (int i = 2; ok && i < n_loads; ++i) {
                     if (!CAUSAL && me == 0 && i == take_at) {
                         next_w = take_item();
                         taken = true;
@@ -329,7 +408,7 @@ __global__ void __launch_bounds__(384, 1)
                     ok = issue_kv(i);
                 }
                 if (!CAUSAL && me == 0 && !taken) next_w = take_item();
-                g += 2 * item.nk1;
+                g += n_loads;
             }
             // Every load of this CTA is issued: the next kernel in the stream may be
             // scheduled (it waits for this grid's completion before reading memory).
@@ -356,10 +435,14 @@ __global__ void __launch_bounds__(384, 1)
                 const int w = CAUSAL ? fwd_work_index(r) : read_item(r);
                 if (w < 0) { ok = false; break; }
                 if (w >= p.n_items) break;
-                const FwdItem item = fwd_item<CAUSAL>(p, w);
+                const FwdItem item = fwd_item<CAUSAL, SPLIT>(p, w);
                 const int nk = t ? item.nk1 : item.nk0;
+                // loads this tile alone uses: tile 1's extra key tile, and every load
+                // of a split item; the other tile's release is given by hand
+                auto single = [&](int jj) { return SPLIT || (t == 1 && jj >= item.nk0); };
                 for (int j = 0; j <= nk; ++j) {
-                    const int ik = g + 2 * j, iv = g + 2 * j - 1;
+                    const int ik = SPLIT ? g + (j < nk ? fwd_load_index(item, t, j, false) : 0) : g + 2 * j;
+                    const int iv = SPLIT ? g + (j > 0 ? fwd_load_index(item, t, j - 1, true) : 0) : g + 2 * j - 1;
                     if (j == 0) {
                         ok = mbar_wait(&q_full[t], it & 1, abort_flag) &&
                              mbar_wait(&slot_full[ik % SLOTS], (ik / SLOTS) & 1, abort_flag);
@@ -393,7 +476,7 @@ __global__ void __launch_bounds__(384, 1)
                         ++np;
                         if (j >= nk) {
                             tc_commit(&o_done[t]);
-                            if (t == 1 && j - 1 >= item.nk0) mbar_arrive(&slot_empty[iv % SLOTS]);  // tile-1-only load
+                            if (single(j - 1)) mbar_arrive(&slot_empty[iv % SLOTS]);
                             tc_commit(&slot_empty[iv % SLOTS]);
                             break;
                         }
@@ -412,14 +495,14 @@ __global__ void __launch_bounds__(384, 1)
                     // S first; each commit covers every earlier MMA of this thread.
                     if (j > 0) {
                         tc_commit(&o_done[t]);
-                        if (t == 1 && j - 1 >= item.nk0) mbar_arrive(&slot_empty[iv % SLOTS]);  // tile-1-only load
+                        if (single(j - 1)) mbar_arrive(&slot_empty[iv % SLOTS]);
                         tc_commit(&slot_empty[iv % SLOTS]);
                     }
-                    if (t == 1 && j >= item.nk0) mbar_arrive(&slot_empty[ik % SLOTS]);  // tile-1-only load
+                    if (single(j)) mbar_arrive(&slot_empty[ik % SLOTS]);
                     tc_commit(&slot_empty[ik % SLOTS]);
                     if (j == nk - 1) tc_commit(&q_empty[t]);  // Q_t buffer free once this S is done
                 }
-                g += 2 * item.nk1;
+                g += SPLIT ? fwd_item_loads(item) : 2 * item.nk1;
             }
             // Every MMA must be complete before TMEM is released.
             tc_commit(&drain[t]);
@@ -435,15 +518,16 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t o_addr = s_addr + 128;
         const float c2 = p.scale_log2;
         bool ok = true;
-        uint32_t ns = 0, nturn = 0, npv = 0;  // phases consumed so far, counted across items
+        uint32_t ns = 0, nturn = 0, npv = 0, nmerge = 0;  // phases consumed so far, counted across items
         for (int r = 0; ok; ++r) {
             const int w = CAUSAL ? fwd_work_index(r) : read_item_warp(r);
             if (w < 0) { ok = false; break; }
             if (w >= p.n_items) break;
-            const FwdItem item = fwd_item<CAUSAL>(p, w);
+            const FwdItem item = fwd_item<CAUSAL, SPLIT>(p, w);
             const int nk = t ? item.nk1 : item.nk0;
-            const int grow = item.qb * 2 * BM + t * BM + row;
-            const int q128 = 2 * item.qb + t;  // index of this query tile in 128-row units
+            const int kb = (SPLIT && t) ? item.kb1 : 0;  // first key tile of this query tile
+            const int grow = (SPLIT ? item.row0[t] : item.qb * 2 * BM + t * BM) + row;
+            const int q128 = 2 * item.qb + t;  // index of this query tile in 128-row units (causal)
             float m_used = -INFINITY, l = 0.f;
             for (int j = 0; j < nk; ++j) {
                 const bool w1 = mbar_wait(&s_full[t], ns & 1, abort_flag);
@@ -453,7 +537,7 @@ __global__ void __launch_bounds__(384, 1)
                 // valid key columns of this tile for this row: [0, lim)
                 int lim = BN;
                 if (CAUSAL && j == q128) lim = row + 1;
-                if (!CAUSAL && j * BN + BN > p.N) lim = p.N - j * BN;
+                if (!CAUSAL && (kb + j) * BN + BN > p.N) lim = p.N - (kb + j) * BN;
                 // pass 1: row max
                 float mx = -INFINITY;
 #pragma unroll
@@ -556,9 +640,49 @@ __global__ void __launch_bounds__(384, 1)
             const bool w2 = mbar_wait(&o_done[t], (npv - 1) & 1, abort_flag);
             if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
             tc_fence_after();
-            const float inv_l = 1.f / l;
+            // Split item: tile 0 hands this row's max and sum to tile 1 (through
+            // its own staging buffer, whose last bulk store has read it) and leaves
+            // O_0 in TMEM; tile 1 merges the two partial results, O = (O_0 l_0 2^(m_0-M)
+            // + O_1 l_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M)) with M = max(m_0, m_1),
+            // as for two blocks of keys of the online softmax, and frees both O regions.
+            float2* xch = reinterpret_cast<float2*>(sO + quad * C::STAGE_O_BYTES);
+            if (SPLIT && t == 0) {
+                if (lane == 0) bulk_wait_read_all();
+                __syncwarp();
+                xch[lane] = make_float2(m_used, l);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(merge_bar);
+                continue;
+            }
+            float m_fin = m_used, l_fin = l;
+            if (SPLIT) {
+                const bool wm = mbar_wait(merge_bar, nmerge & 1, abort_flag);
+                ++nmerge;
+                if (!__all_sync(0xffffffffu, wm)) { ok = false; break; }
+                tc_fence_after();
+                const float2 ml0 = xch[lane];
+                m_fin = fmaxf(ml0.x, m_used);
+                const float a0 = ex2_approx(ml0.x - m_fin), a1 = ex2_approx(m_used - m_fin);
+                l_fin = ml0.y * a0 + l * a1;
+                // O_1 <- O_1 2^(m_1-M) + O_0 2^(m_0-M), in TMEM; O_0 is then free
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r3[32], r4[32];
+                    tmem_ld32(o_addr + c * 32, r3);
+                    tmem_ld32(o_addr - 256 + c * 32, r4);  // tile 0's O, same lanes
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        r3[i] = __float_as_uint(__uint_as_float(r3[i]) * a1 + __uint_as_float(r4[i]) * a0);
+                    tmem_st32(o_addr + c * 32, r3);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&o_free[0]);
+            }
+            const float inv_l = 1.f / l_fin;
             uint8_t* stage = sO + warp * C::STAGE_O_BYTES;
-            const int row0 = item.qb * 2 * BM + t * BM + quad * 32;  // first row of this warp
+            const int row0 = (SPLIT ? item.row0[t] : item.qb * 2 * BM + t * BM) + quad * 32;  // first row of this warp
             if constexpr (F32OUT) {
                 // fp32 O, 32 columns (128 bytes of a row) at a time; chunk i of row
                 // r sits at slot i ^ (r & 7) of the staging buffer
@@ -631,7 +755,7 @@ __global__ void __launch_bounds__(384, 1)
             }
             }
             if (grow < p.N)
-                p.lse[static_cast<size_t>(item.bh) * p.N + grow] = (m_used + log2f(l)) * 0.69314718055994530942f;
+                p.lse[static_cast<size_t>(item.bh) * p.N + grow] = (m_fin + log2f(l_fin)) * 0.69314718055994530942f;
         }
         // the bulk stores read the staging buffers: complete before the CTA exits
         if (!F32OUT && lane == 0) bulk_wait_all();

@@ -36,10 +36,12 @@
  *    device memory, so the stream's order of memory effects is unchanged.
  *  - Calls may be captured in CUDA graphs. A non-causal attn_fwd (and
  *    attn_fwd_f16, attn_fwd_f32) hands out its work items through one of 64
- *    device counters, taken by successive calls in turn and back at zero when
- *    the call's kernel ends: at most 64 such calls may be in flight at once,
- *    and a captured call keeps its counter at every replay, so replays of one
- *    graph must not run concurrently with each other.
+ *    device counters, taken by successive launches in turn and back at zero when
+ *    the launch's kernel ends; a call whose last round of query blocks would
+ *    leave most SMs idle makes two launches (the second, in 128-row halves,
+ *    right behind the first) and takes two counters: at most 32 such calls may
+ *    be in flight at once, and a captured call keeps its counters at every
+ *    replay, so replays of one graph must not run concurrently with each other.
  */
 #ifndef EXACT_ATTENTION_RING_B200_ATTN_H
 #define EXACT_ATTENTION_RING_B200_ATTN_H

@@ -182,6 +182,28 @@ def test_repeatable_large_logits_many_tiles():
         assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_split_last_round(d):
+    """A non-causal problem whose last round holds at most half as many query
+    blocks as there are SMs runs that round as a second launch of 128-row items,
+    each tile of a CTA over half of the keys, merged in the epilogue. B1 H32
+    N1536: 192 blocks, so on 148 SMs the first launch takes 148 and the split
+    launch the other 44 (88 items). Every row against the oracle."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    blocks = 32 * 1536 // 256
+    assert 2 * (blocks % sms) <= sms, "shape chosen for a split last round on this GPU"
+    check_full(1, 32, 32, 1536, d, False, 6300 + d)
+
+
+def test_split_last_round_ragged_odd_key_tiles():
+    """Split items with an odd number of key tiles (tile 1 takes the extra one,
+    with no turn) and a ragged last key tile in tile 1's half: N = 1100 gives
+    nine key tiles, 4 for tile 0 and 5 for tile 1; B1 H8 gives 40 blocks, all
+    split."""
+    check_full(1, 8, 8, 1100, 128, False, 6350)
+    check_full(1, 8, 2, 1100, 64, False, 6351)
+
+
 def test_work_counter_slots_are_reused_and_reset():
     """Non-causal launches hand out work items from a per-launch counter slot
     that the launch's last CTA resets. 70 launches in a row (more than the 64
