@@ -74,8 +74,10 @@ NCU_TRAFFIC = {
     "decode": {"bytes_per_launch": 536959744 + 3461376, "source_sha": "eaaf414296e5590d"},
     "decode_b1_l32k": {"bytes_per_launch": 134302976 + 3129856, "source_sha": "eaaf414296e5590d"},
     "decode_b8_l32k": {"bytes_per_launch": 1073927168 + 3971072, "source_sha": "eaaf414296e5590d"},
-    "attn_fwd_causal": {"bytes_per_launch": 131980800 + 12869120, "source_sha": "7eb65e92f430f85e"},
-    "attn_fwd_noncausal": {"bytes_per_launch": 100789760 + 13249536, "source_sha": "7eb65e92f430f85e"},
+    "attn_fwd_causal": {"bytes_per_launch": 135730176 + 13396224, "source_sha": "4a0ebecc98b69899"},
+    # the non-causal call is two launches at this shape (the plain kernel, then the last round in
+    # 128-row halves): their sum
+    "attn_fwd_noncausal": {"bytes_per_launch": 87890176 + 8552704 + 13959936 + 5120, "source_sha": "4a0ebecc98b69899"},
 }
 
 
@@ -228,6 +230,56 @@ def measure_extra_paths(eab, q, k, v, o, lse, p, flush_l2, stream, iters=10, war
     torch.cuda.synchronize()
     assert eab.attn_device_status() == 0
     return t_bwd, t_fp8, t_quant
+
+
+def fwd_launch_count(B, Hq, N, causal, sms):
+    """Kernel launches of one attn_fwd call: two for a non-causal problem whose
+    last round of 256-row query blocks holds at most half as many blocks as
+    there are SMs (and N spans two key tiles), whose tail runs as a second
+    launch in 128-row halves; else one."""
+    if causal:
+        return 1
+    rem = (B * Hq * ((N + 255) // 256)) % sms
+    return 2 if ((N + 127) // 128 >= 2 and rem > 0 and 2 * rem <= sms) else 1
+
+
+# Causal d = 128 prefill at the longer shapes of the sequence sweep and at the
+# grouped-query shapes (B, Hq, Hkv, N): timed alone after the step like the
+# extra paths, so that the bench line carries the causal rate beyond N = 2048.
+CAUSAL_SWEEP = [(4, 16, 16, 4096), (2, 16, 16, 8192), (1, 16, 16, 16384), (1, 32, 8, 8192), (1, 32, 1, 8192)]
+
+
+def measure_causal_sweep(eab, flush_l2, stream, tc_peak, iters=10, warm=3, seed=4242):
+    out = []
+    gen = torch.Generator(device="cuda")
+    for (B, Hq, Hkv, N) in CAUSAL_SWEEP:
+        d = 128
+        gen.manual_seed(seed + N + Hkv)
+        q = torch.randn(B, Hq, N, d, device="cuda", generator=gen).to(torch.bfloat16)
+        k = torch.randn(B, Hkv, N, d, device="cuda", generator=gen).to(torch.bfloat16)
+        v = torch.randn(B, Hkv, N, d, device="cuda", generator=gen).to(torch.bfloat16)
+        o = torch.empty_like(q)
+        lse = torch.empty(B, Hq, N, device="cuda")
+        fn = lambda: eab.attn_fwd(q, k, v, o, lse, True, d ** -0.5, stream)
+        for _ in range(warm):
+            fn()
+        ts = []
+        for _ in range(iters):
+            flush_l2()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ms = sorted(ts)[len(ts) // 2]
+        tf = 2.0 * B * Hq * N * N * d / (ms * 1e-3) / 1e12
+        out.append({"workload": f"B{B} Hq{Hq} Hkv{Hkv} N{N} d{d} causal", "ms": round(ms, 5),
+                    "tflops": round(tf, 1), "frac": round(tf / tc_peak, 4)})
+        del q, k, v, o, lse
+    torch.cuda.synchronize()
+    assert eab.attn_device_status() == 0
+    return out
 
 
 def run_ours(args):
@@ -397,6 +449,7 @@ def run_ours(args):
     # ---- roofline of each kernel; the dominant one goes in "roofline"
     tc_peak = peaks["bf16_tflops"]
     hbm_peak = peaks["hbm_gbs"]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     fwd_sha = kernel_sha("attn_fwd_sm100.cuh")
     dec_sha = kernel_sha("decode_sm100.cuh")
     def traffic(name, sha):
@@ -406,7 +459,10 @@ def run_ours(args):
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": round(tflops_c / tc_peak, 4),
                 "traffic": traffic("attn_fwd_causal", fwd_sha), "ms": round(t_fwd_c, 5),
                 "peak_source": f"{peak_src} bf16_tflops (burst)"}
-    roof_fwd_nc = {"kernel": "attn_fwd_kernel<128,noncausal>", "bound": "tensor", "achieved": round(tflops_n, 1),
+    nc_launches = fwd_launch_count(p.B, p.Hq, p.N, False, sms)
+    roof_fwd_nc = {"kernel": "attn_fwd_kernel<128,noncausal>" + (" and its split last round (two launches, one "
+                                                                  "event interval)" if nc_launches == 2 else ""),
+                   "bound": "tensor", "achieved": round(tflops_n, 1),
                    "peak": tc_peak, "unit": "TFLOP/s", "frac": round(tflops_n / tc_peak, 4),
                    "traffic": traffic("attn_fwd_noncausal", fwd_sha), "ms": round(t_fwd_n, 5)}
     dec_roofs = {}
@@ -451,6 +507,13 @@ def run_ours(args):
             }
         except Exception as exc:  # the headline line is printed regardless
             extra = {"error": f"{type(exc).__name__}: {exc}"}
+        try:
+            extra["prefill_causal_d128"] = {
+                "note": "sequence-sweep and grouped-query shapes, bf16 N(0,1) drawn on the device; timed alone "
+                        "after the step, L2 flushed before each launch, median of 10",
+                "shapes": measure_causal_sweep(eab, flush_l2, stream, tc_peak)}
+        except Exception as exc:
+            extra["prefill_causal_d128"] = {"error": f"{type(exc).__name__}: {exc}"}
 
     cpu = cpu_baseline_sample(budget_s=args.cpu_budget) if (rank == 0 and world == 1 and not args.no_cpu) else None
 
@@ -492,7 +555,7 @@ def run_ours(args):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
                     "pipeline": "per step: H2D of q,k,v, attn_fwd, D2H of o,lse; copies on their own streams, "
                                 "so step i's kernel overlaps step i+1's input copy and step i-1's output copy"},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": (3 + fwd_launch_count(p.B, p.Hq, p.N, False, sms)) * args.steps,
             "extra_paths": extra,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,

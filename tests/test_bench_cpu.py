@@ -30,3 +30,16 @@ def test_profile_subcommand_parses():
                          capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stderr
     assert "--causal" in out.stdout
+
+
+def test_launch_count_follows_the_split_rule():
+    """The step's launch count: a non-causal call whose last round holds at most
+    half as many 256-row query blocks as SMs makes a second launch."""
+    b = _bench()
+    assert b.fwd_launch_count(2, 32, 2048, True, 148) == 1
+    assert b.fwd_launch_count(2, 32, 2048, False, 148) == 2   # 512 blocks: last round 68 <= 74
+    assert b.fwd_launch_count(8, 16, 2048, False, 148) == 1   # 1024 blocks: last round 136 > 74
+    assert b.fwd_launch_count(1, 37, 1024, False, 148) == 1   # 148 blocks: no last round
+    assert b.fwd_launch_count(1, 1, 128, False, 148) == 1     # one key tile: nothing to split
+    assert b.fwd_launch_count(1, 1, 256, False, 148) == 2     # one block, two key tiles
+    assert len(b.CAUSAL_SWEEP) >= 3
