@@ -251,7 +251,9 @@ template <int D, bool CAUSAL>
 attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
     const long long rows = static_cast<long long>(p.B) * p.Hq * p.N;
-    launch_pdl(bwd_delta_kernel<D>, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, stream, p, rows);
+    constexpr long long kRowsPerBlock = 256 / (D / 8);
+    launch_pdl(bwd_delta_kernel<D>, dim3(static_cast<unsigned>((rows + kRowsPerBlock - 1) / kRowsPerBlock)), dim3(256),
+               0, stream, p, rows);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     attn_status_t st = launch_bwd_tile<D, CAUSAL, true>(tk, tv, tq, tdo, p, stream);
     if (st != ATTN_OK) return st;

@@ -66,23 +66,30 @@ struct BwdCfg {
     static constexpr uint32_t TMEM_COLS = 512;
 };
 
-// Delta_i = sum_t dO_it O_it, one warp per row.
+// Delta_i = sum_t dO_it O_it: D / 8 threads per row, each with one 16-byte load
+// of dO and of O (8 elements), the partial sums reduced across those threads.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdParams p, long long rows) {
     grid_dep_wait();  // the previous kernel's writes are visible from here on
     grid_dep_launch();
-    const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    if (row >= rows) return;
-    const int lane = threadIdx.x & 31;
-    constexpr int CPL = D / 32;
-    const __nv_bfloat16* a = p.dout + row * D + lane * CPL;
-    const __nv_bfloat16* b = p.o + row * D + lane * CPL;
+    constexpr int TPR = D / 8;  // threads per row (16 or 8)
+    const long long row = static_cast<long long>(blockIdx.x) * (256 / TPR) + threadIdx.x / TPR;
+    const int part = threadIdx.x % TPR;
     float acc = 0.f;
+    if (row < rows) {
+        const uint4 a = *reinterpret_cast<const uint4*>(p.dout + row * D + part * 8);
+        const uint4 b = *reinterpret_cast<const uint4*>(p.o + row * D + part * 8);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) acc += __bfloat162float(a[i]) * __bfloat162float(b[i]);
+        for (int i = 0; i < 4; ++i) {
+            const float2 af = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[i]));
+            const float2 bf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw[i]));
+            acc += af.x * bf.x + af.y * bf.y;
+        }
+    }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) p.delta[row] = acc;
+    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (row < rows && part == 0) p.delta[row] = acc;
 }
 
 // Shared skeleton of the two tile kernels. One block owns a fixed pair of
