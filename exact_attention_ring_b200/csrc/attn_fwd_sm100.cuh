@@ -642,9 +642,10 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_after();
             // Split item: tile 0 hands this row's max and sum to tile 1 (through
             // its own staging buffer, whose last bulk store has read it) and leaves
-            // O_0 in TMEM; tile 1 merges the two partial results, O = (O_0 l_0 2^(m_0-M)
-            // + O_1 l_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M)) with M = max(m_0, m_1),
-            // as for two blocks of keys of the online softmax, and frees both O regions.
+            // its accumulator A_0 (the unnormalised sum of p v) in TMEM; tile 1
+            // merges the two as the online softmax merges two blocks of keys,
+            // O = (A_0 2^(m_0-M) + A_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M)) with
+            // M = max(m_0, m_1), and frees A_0's columns once it has read them.
             float2* xch = reinterpret_cast<float2*>(sO + quad * C::STAGE_O_BYTES);
             if (SPLIT && t == 0) {
                 if (lane == 0) bulk_wait_read_all();
@@ -664,7 +665,7 @@ __global__ void __launch_bounds__(384, 1)
                 m_fin = fmaxf(ml0.x, m_used);
                 const float a0 = ex2_approx(ml0.x - m_fin), a1 = ex2_approx(m_used - m_fin);
                 l_fin = ml0.y * a0 + l * a1;
-                // O_1 <- O_1 2^(m_1-M) + O_0 2^(m_0-M), in TMEM; O_0 is then free
+                // A_1 <- A_1 2^(m_1-M) + A_0 2^(m_0-M), in TMEM; A_0 is then free
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t r3[32], r4[32];
