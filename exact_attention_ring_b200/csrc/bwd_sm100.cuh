@@ -176,7 +176,13 @@ __global__ void __launch_bounds__(320, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    grid_dep_wait();  // the previous kernel's writes are visible from here on
+    // The dK/dV kernel waits for the previous kernel (Delta) here. The dQ kernel
+    // reads nothing the dK/dV kernel writes, and it is scheduled only once every
+    // dK/dV block has passed its own wait (its trigger follows it), so Delta is
+    // complete by then: its blocks start on the SMs the dK/dV tail frees and wait
+    // for the dK/dV grid only before they exit, which keeps the stream's order
+    // of completion.
+    if (DKDV) grid_dep_wait();
 
     // plane (batch * heads + head) and tile row of streamed step s
     auto step_src = [&](int s, int* plane, int* trow) {
@@ -460,6 +466,7 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
+    if (!DKDV) grid_dep_wait();
 }
 
 }  // namespace eab
