@@ -32,7 +32,9 @@
 // while the second half is computed. The next step's dP^T MMAs are issued
 // after the accumulating MMAs that read P^T / dS^T from its columns, so the
 // tensor pipe's issue order keeps them intact until read (as in the forward
-// pass). Every wait is bounded.
+// pass). Every wait is bounded. The dQ kernel needs nothing the dK/dV kernel
+// writes: its blocks start as the dK/dV tail frees SMs and wait for that grid
+// only before they exit.
 #pragma once
 
 #include "sm100_ptx.cuh"
