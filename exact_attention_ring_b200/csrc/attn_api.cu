@@ -135,6 +135,7 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
         return ATTN_ERR_CUDA;
     FwdParams p = p0;
     p.block0 = 0;
+    p.chained = 0;
     if constexpr (!CAUSAL) {
         // Non-causal items all cost the same, so a last round of r <= SMs/2 query
         // blocks would leave most CTAs idle for a whole item. Those blocks go to a
@@ -152,6 +153,7 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                 if (st != ATTN_OK) return st;
             }
             p.block0 = n_full;
+            p.chained = n_full > 0 ? 1 : 0;
             p.n_items = 2 * rem;
             p.sched_slot = next_fwd_slot();
             return launch_fwd_kernel<D, CAUSAL, F32OUT, E, true>(tq, tk, tv, to, p, p.n_items, stream);

@@ -74,6 +74,7 @@ struct FwdParams {
     int n_qblocks;     // ceil(N / 256)
     int n_items;       // work items of this launch
     int block0;        // split launches: the first query block; item w is half w & 1 of block block0 + w / 2
+    int chained;       // split launches: 1 when the launch of the call's other blocks precedes this one
     float scale_log2;  // scale * log2(e)
     int sched_slot;    // this launch's work counter in g_fwd_sched
 };
@@ -299,7 +300,14 @@ __global__ void __launch_bounds__(384, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    grid_dep_wait();  // the previous kernel's writes are visible from here on
+    // The previous kernel's writes are visible after this wait. A split launch
+    // that follows the launch of the same call's other blocks does not read
+    // their outputs, and it is scheduled only once every block of that launch
+    // has passed this wait (their trigger follows it), so its inputs are
+    // complete: its blocks start on the SMs that launch's tail frees and wait
+    // for it only before they exit, which keeps the stream's order of completion.
+    const bool wait_at_end = SPLIT && p.chained;
+    if (!wait_at_end) grid_dep_wait();
 
     // Work item r of this CTA: published by the first producer's thread (the
     // first item is the CTA's index, later ones come from the launch's counter,
@@ -768,6 +776,7 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
+    if (wait_at_end) grid_dep_wait();
     // Every item this CTA took has been taken; the last CTA to get here resets the
     // launch's counter slot (no CTA of this launch reads it any more).
     if (!CAUSAL && threadIdx.x == 0) {

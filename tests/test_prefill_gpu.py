@@ -204,6 +204,32 @@ def test_split_last_round_ragged_odd_key_tiles():
     check_full(1, 8, 2, 1100, 64, False, 6351)
 
 
+@pytest.mark.parametrize("shape", [(2, 32, 2048), (1, 8, 1100)], ids=["two_launches", "split_only"])
+def test_split_launch_stream_order(shape):
+    """The split launch of a non-causal call starts its blocks in the tail of
+    the call's first launch and waits for it only before it exits; a split
+    launch with no first launch waits for the previous kernel at its start.
+    Inputs written by the kernel just before the call, and a copy of the
+    outputs made by the kernel just after it, must see the stream's order."""
+    B, H, N = shape
+    d = 128
+    q, k, v = (t.to(DEV) for t in si.make_qkv(6400 + N, B, H, H, N, d))
+    o_ref, lse_ref = eab.attention(q, k, v, causal=False)
+    torch.cuda.synchronize()
+    q_in = torch.full_like(q, float("nan"))
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full((B, H, N), float("nan"), device=DEV)
+    for _ in range(3):
+        q_in.fill_(float("nan"))
+        o.fill_(float("nan"))
+        q_in.copy_(q)  # written by the kernel right before the call
+        eab.attn_fwd(q_in, k, v, o, lse, False, d ** -0.5)
+        o_after, lse_after = o.clone(), lse.clone()  # read by the kernel right after it
+        torch.cuda.synchronize()
+        assert eab.attn_device_status() == 0
+        assert torch.equal(o_after, o_ref) and torch.equal(lse_after, lse_ref)
+
+
 def test_work_counter_slots_are_reused_and_reset():
     """Non-causal launches hand out work items from a per-launch counter slot
     that the launch's last CTA resets. 70 launches in a row (more than the 64
