@@ -105,7 +105,7 @@ struct FwdCfg {
     static constexpr int ITEM_RING = 4;  // work items handed from the fetching thread to the other roles
     // q_full, q_empty, slot_full, slot_empty, s_full, p_full, o_done, o_free, turn, drain, p_half,
     // item_full, item_empty, merge
-    static constexpr int NUM_BARRIERS = 2 * 2 + 2 * SLOTS + 7 * 2 + 2 * ITEM_RING + 1;
+    static constexpr int NUM_BARRIERS = 2 * 2 + 2 * (SLOTS + 1) + 7 * 2 + 2 * ITEM_RING + 1;
     // item readers: the second producer, the two MMA issuers and the eight softmax warps
     static constexpr int ITEM_READERS = 11;
     static constexpr int SMEM_BYTES = 1024 + TILES * Q_TILE_BYTES + SLOTS * TILE_BYTES + 8 * STAGE_O_BYTES +
@@ -241,12 +241,19 @@ __global__ void __launch_bounds__(384, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     const FwdParams p) {
     using C = FwdCfg<D>;
-    constexpr int BM = C::BM, BN = C::BN, SLOTS = C::SLOTS;
+    constexpr int BM = C::BM, BN = C::BN;
+    // split launches: both query tiles read Q buffer 0, and Q buffer 1 is a fifth
+    // ring slot (a split item's K/V tiles each serve one tile: four loads a step)
+    constexpr int SLOTS = C::SLOTS + (SPLIT ? 1 : 0);
+    static_assert(C::Q_TILE_BYTES == C::TILE_BYTES, "the extra slot is a Q buffer");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
     uint8_t* sKV = smem + C::TILES * C::Q_TILE_BYTES;
-    uint8_t* sO = sKV + SLOTS * C::TILE_BYTES;  // [8 warps][32 rows][64 bf16] epilogue staging
+    uint8_t* sO = sKV + C::SLOTS * C::TILE_BYTES;  // [8 warps][32 rows][64 bf16] epilogue staging
+    auto slot_ptr = [&](int slot) -> uint8_t* {
+        return slot < C::SLOTS ? sKV + slot * C::TILE_BYTES : sQ + C::Q_TILE_BYTES;
+    };
     uint64_t* bars = reinterpret_cast<uint64_t*>(sO + 8 * C::STAGE_O_BYTES);
     uint64_t* q_full = bars;                   // [2] Q tile t loaded
     uint64_t* q_empty = q_full + 2;            // [2] last S of Q tile t's buffer done
@@ -373,7 +380,7 @@ __global__ void __launch_bounds__(384, 1)
                     int kt = i >> 1;
                     const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;
                     if constexpr (SPLIT) tm = fwd_load_kind(item, i, &kt) ? &tm_v : &tm_k;
-                    uint8_t* dst = sKV + slot * C::TILE_BYTES;
+                    uint8_t* dst = slot_ptr(slot);
 #pragma unroll
                     for (int c = 0; c < C::CHUNKS; ++c) {
                         if ((gi * C::CHUNKS + c) % C::NUM_PRODUCERS != me) continue;
@@ -384,6 +391,7 @@ __global__ void __launch_bounds__(384, 1)
                 };
                 // issue (this producer's boxes of) Q tile t of the item
                 auto issue_q = [&](int t) -> bool {
+                    if (SPLIT && t == 1) return true;  // tile 1 reads Q buffer 0
                     bool any = false;
 #pragma unroll
                     for (int c = 0; c < C::CHUNKS; ++c) any |= ((t * C::CHUNKS + c) % C::NUM_PRODUCERS) == me;
@@ -424,7 +432,7 @@ __global__ void __launch_bounds__(384, 1)
             // Let every copy in flight land before the CTA can exit.
             if (it > 0) {
                 mbar_wait(&q_full[0], (it - 1) & 1, nullptr);
-                mbar_wait(&q_full[1], (it - 1) & 1, nullptr);
+                if (!SPLIT) mbar_wait(&q_full[1], (it - 1) & 1, nullptr);
             }
             for (int i = max(0, g - SLOTS); i < g; ++i) mbar_wait(&slot_full[i % SLOTS], (i / SLOTS) & 1, nullptr);
         }
@@ -435,7 +443,11 @@ __global__ void __launch_bounds__(384, 1)
             constexpr uint32_t idesc_qk = make_idesc(BM, BN, 0, 0, E::fmt);
             constexpr uint32_t idesc_pv = make_idesc(BM, D, 0, 1, E::fmt);
             const uint32_t s_tmem = tmem + t * 256, o_tmem = s_tmem + 128;
-            const uint32_t q_addr = smem_addr(sQ + t * C::Q_TILE_BYTES), kv_addr = smem_addr(sKV);
+            const int tq = SPLIT ? 0 : t;  // the Q buffer this tile reads
+            const uint32_t q_addr = smem_addr(sQ + tq * C::Q_TILE_BYTES), kv_addr = smem_addr(sKV);
+            auto slot_addr = [&](int slot) -> uint32_t {
+                return slot < C::SLOTS ? kv_addr + slot * C::TILE_BYTES : smem_addr(sQ + C::Q_TILE_BYTES);
+            };
             bool ok = true;
             int g = 0;        // K/V load index of the item's K_0
             uint32_t np = 0;  // P_t handed over so far (p_full phases)
@@ -452,7 +464,7 @@ __global__ void __launch_bounds__(384, 1)
                     const int ik = SPLIT ? g + (j < nk ? fwd_load_index(item, t, j, false) : 0) : g + 2 * j;
                     const int iv = SPLIT ? g + (j > 0 ? fwd_load_index(item, t, j - 1, true) : 0) : g + 2 * j - 1;
                     if (j == 0) {
-                        ok = mbar_wait(&q_full[t], it & 1, abort_flag) &&
+                        ok = mbar_wait(&q_full[tq], it & 1, abort_flag) &&
                              mbar_wait(&slot_full[ik % SLOTS], (ik / SLOTS) & 1, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
@@ -467,7 +479,7 @@ __global__ void __launch_bounds__(384, 1)
                              mbar_wait_spin(&p_half[t], np & 1, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
-                        const uint32_t v_addr = kv_addr + (iv % SLOTS) * C::TILE_BYTES;
+                        const uint32_t v_addr = slot_addr(iv % SLOTS);
 #pragma unroll
                         for (int kk = 0; kk < BN / 16; ++kk) {
                             if (kk == BN / 32) {
@@ -490,7 +502,7 @@ __global__ void __launch_bounds__(384, 1)
                         }
                     }
                     // S_t(j) = Q_t K_j^T
-                    const uint32_t k_addr = kv_addr + (ik % SLOTS) * C::TILE_BYTES;
+                    const uint32_t k_addr = slot_addr(ik % SLOTS);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t koff = (kk & 3) * 32;  // 16 elements = 32 bytes inside the swizzle row
@@ -508,7 +520,9 @@ __global__ void __launch_bounds__(384, 1)
                     }
                     if (single(j)) mbar_arrive(&slot_empty[ik % SLOTS]);
                     tc_commit(&slot_empty[ik % SLOTS]);
-                    if (j == nk - 1) tc_commit(&q_empty[t]);  // Q_t buffer free once this S is done
+                    // Q_t's buffer is free once this S is done (split launches take one
+                    // item per CTA: their Q buffer is never reloaded)
+                    if (j == nk - 1 && !(SPLIT && t == 1)) tc_commit(&q_empty[t]);
                 }
                 g += SPLIT ? fwd_item_loads(item) : 2 * item.nk1;
             }
