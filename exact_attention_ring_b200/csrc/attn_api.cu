@@ -243,7 +243,7 @@ attn_status_t launch_bwd_tile(const CUtensorMap& fa, const CUtensorMap& fb, cons
     auto kern = bwd_tile_kernel<D, CAUSAL, DKDV>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
-    const dim3 grid((p.N + C::BT - 1) / C::BT, p.B * (DKDV ? p.Hkv : p.Hq));
+    const dim3 grid(p.B * (DKDV ? p.Hkv : p.Hq), (p.N + C::BT - 1) / C::BT);
     if (launch_pdl(kern, grid, dim3(C::NUM_THREADS), C::SMEM_BYTES, stream, fa, fb, sa, sb, p) != cudaSuccess)
         return ATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -397,7 +397,8 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
     if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || (causal != 0 && causal != 1) || !scale_ok(scale))
         return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-    if (static_cast<long long>(B) * Hq > 65535LL) return ATTN_ERR_INVALID_ARG;
+    // the tile kernels' grid is (planes, 128-row tiles): both within 65535
+    if (static_cast<long long>(B) * Hq > 65535LL || (N + 127) / 128 > 65535) return ATTN_ERR_INVALID_ARG;
     if ((static_cast<long long>(B) * Hq * N + 7) / 8 > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
     CUtensorMap tq, tk, tv, tdo;
     if (!make_map<ElemBf16>(&tq, q, d, N, B * Hq, 128) || !make_map<ElemBf16>(&tk, k, d, N, B * Hkv, 128) ||

@@ -141,12 +141,14 @@ __global__ void __launch_bounds__(320, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.Hq / p.Hkv;
     const int n_tiles = (p.N + BT - 1) / BT;
-    // the fixed tile: key tile (dK/dV) or query tile (dQ); under the causal
-    // mask the blocks with the most steps are launched first
-    const int tile = (DKDV || !CAUSAL) ? blockIdx.x : n_tiles - 1 - blockIdx.x;
+    // the fixed tile: key tile (dK/dV) or query tile (dQ). The grid is (planes,
+    // tiles) and blocks start in the order of their linear index, planes
+    // fastest: under the causal mask every plane's block with the most steps
+    // starts before any block with fewer, so the last wave holds the shortest.
+    const int tile = (DKDV || !CAUSAL) ? blockIdx.y : n_tiles - 1 - blockIdx.y;
     // fixed head (KV head for dK/dV, query head for dQ) and its batch
-    const int b = blockIdx.y / (DKDV ? p.Hkv : p.Hq);
-    const int hfix = blockIdx.y % (DKDV ? p.Hkv : p.Hq);
+    const int b = blockIdx.x / (DKDV ? p.Hkv : p.Hq);
+    const int hfix = blockIdx.x % (DKDV ? p.Hkv : p.Hq);
     // the streamed steps: dK/dV walks (query head of the group, query tile);
     // dQ walks key tiles. Causal: query tile >= key tile.
     const int t_lo = DKDV ? (CAUSAL ? tile : 0) : 0;
