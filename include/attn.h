@@ -180,11 +180,12 @@ attn_status_t attn_merge(float* o_acc, float* lse_acc, const float* o_blk, const
  *  delta      [B, Hq, N]     fp32 (device): workspace, overwritten with Delta
  *  dq         [B, Hq, N, d]  bf16 (device, written)
  *  dk, dv     [B, Hkv, N, d] bf16 (device, written)
- *  B*Hq <= 65535; N >= 1; d 64 or 128 (else ATTN_ERR_UNSUPPORTED); causal 0/1
- *  (query i sees keys j <= i); scale finite and > 0. Outputs must not overlap
- *  the inputs. Three launches on `stream`: Delta, then dk/dv (one block per
- *  128-key tile and key/value head), then dq (one block per 128-row query tile
- *  and query head).
+ *  B*Hq <= 65535; 1 <= N <= 65535 * 128; d 64 or 128 (else
+ *  ATTN_ERR_UNSUPPORTED); causal 0/1 (query i sees keys j <= i); scale finite
+ *  and > 0. Outputs must not overlap the inputs. Three launches on `stream`:
+ *  Delta, then dk/dv (one block per 128-key tile and key/value head), then dq
+ *  (one block per 128-row query tile and query head); under the causal mask the
+ *  blocks with the most work start first.
  */
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                        const void* dout, float* delta, void* dq, void* dk, void* dv,
