@@ -223,8 +223,11 @@ def _bwd(lib, q=16, k=32, v=48, o=64, lse=80, do=96, delta=112, dq=128, dk=144, 
 @pytest.mark.parametrize("kw", [dict(q=0), dict(k=0), dict(v=0), dict(o=0), dict(lse=0), dict(do=0),
                                 dict(delta=0), dict(dq=0), dict(dk=0), dict(dv=0), dict(dq=136), dict(lse=84),
                                 dict(B=0), dict(N=0), dict(Hq=3, Hkv=2), dict(causal=2), dict(scale=0.0),
-                                dict(scale=float("nan")), dict(B=2, Hq=40000, Hkv=40000)])
+                                dict(scale=float("nan")), dict(B=2, Hq=40000, Hkv=40000),
+                                dict(N=65535 * 128 + 1)])
 def test_bwd_rejects_invalid(lib, kw):
+    """Rejected before any device call; the last case is past the tile kernels'
+    65535 tiles of 128 rows."""
     assert _bwd(lib, **kw) == INVALID
 
 
@@ -267,22 +270,3 @@ def test_fwd_fp8_rejects_invalid(lib, kw):
 @pytest.mark.parametrize("d", [64, 96, 256])
 def test_fwd_fp8_rejects_unsupported_head_dim(lib, d):
     assert _fwd8(lib, d=d) == UNSUPPORTED
-
-
-def _bwd(lib, B=1, Hq=2, Hkv=1, N=8, d=64, causal=0, scale=0.125):
-    P = ctypes.c_void_p
-    lib.attn_bwd.restype = ctypes.c_int
-    ptrs = [P(16 * (i + 1)) for i in range(10)]  # q, k, v, o, lse, dout, delta, dq, dk, dv (never dereferenced)
-    return lib.attn_bwd(*ptrs, B, Hq, Hkv, N, d, causal, ctypes.c_float(scale), None)
-
-
-@pytest.mark.parametrize("kw", [dict(B=0), dict(N=0), dict(Hq=3, Hkv=2), dict(causal=2), dict(scale=0.0),
-                                dict(B=65536), dict(N=65535 * 128 + 1)])
-def test_bwd_rejects_invalid(lib, kw):
-    """Rejected before any device call, including grids past 65535 planes or
-    65535 tiles of 128 rows."""
-    assert _bwd(lib, **kw) == INVALID
-
-
-def test_bwd_rejects_unsupported_head_dim(lib):
-    assert _bwd(lib, d=96) == UNSUPPORTED
