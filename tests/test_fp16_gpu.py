@@ -31,6 +31,19 @@ def test_fwd_f16_matches_oracle(B, Hq, Hkv, N, d, causal):
     assert_attn_close(o, lse, o_ref, lse_ref, f"fp16 B{B} Hq{Hq} Hkv{Hkv} N{N} d{d} causal={causal}")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_fwd_f16_split_last_round(d):
+    """fp16 through the two launches of a non-causal call whose last round is
+    split (B1 Hq32 Hkv8 N1536: 192 query blocks, 44 of them split on 148 SMs)."""
+    B, Hq, Hkv, N = 1, 32, 8, 1536
+    q, k, v = si.make_qkv(760 + d, B, Hq, Hkv, N, d, dtype=F16)
+    o, lse = eab.attention(q.to(DEV), k.to(DEV), v.to(DEV), causal=False, scale=d ** -0.5)
+    torch.cuda.synchronize()
+    assert o.dtype == F16 and eab.attn_device_status() == 0
+    o_ref, lse_ref = oracle.attention(q, k, v, False, d ** -0.5)
+    assert_attn_close(o, lse, o_ref, lse_ref, f"fp16 split B{B} Hq{Hq} Hkv{Hkv} N{N} d{d}")
+
+
 def test_fwd_f16_large_logits_sampled():
     """LLaMA-7B shape with Q x 8 (exact in fp16) on sampled rows."""
     B, H, N, d = 2, 32, 2048, 128

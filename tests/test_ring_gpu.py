@@ -78,6 +78,25 @@ def test_merge_init_and_out_paths_are_exact(d):
     assert torch.equal(la2.cpu(), ref_l.cpu())
 
 
+def test_fwd_f32_split_last_round():
+    """attn_fwd_f32 through the two launches of a non-causal call whose last
+    round is split (B1 Hq32 Hkv8 N1536): bf16 of its O is attn_fwd's O bit for
+    bit and the fp32 O is within tolerance of the oracle."""
+    B, Hq, Hkv, N, d = 1, 32, 8, 1536, 128
+    q, k, v = si.make_qkv(4150, B, Hq, Hkv, N, d)
+    qg, kg, vg = q.to(DEV), k.to(DEV), v.to(DEV)
+    scale = d ** -0.5
+    o32 = torch.empty(B, Hq, N, d, device=DEV)
+    l32 = torch.empty(B, Hq, N, device=DEV)
+    eab.attn_fwd_f32(qg, kg, vg, o32, l32, False, scale)
+    o16, l16 = eab.attention(qg, kg, vg, causal=False, scale=scale)
+    torch.cuda.synchronize()
+    assert eab.attn_device_status() == 0
+    assert torch.equal(o32.to(torch.bfloat16), o16) and torch.equal(l32, l16)
+    o_ref, lse_ref = oracle.attention(q, k, v, False, scale)
+    assert_attn_close(o32, l32, o_ref, lse_ref, "fwd_f32 split B1 Hq32 Hkv8 N1536")
+
+
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("N", [1, 130, 300, 2048])
