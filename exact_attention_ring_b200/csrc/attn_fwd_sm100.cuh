@@ -739,12 +739,10 @@ __global__ void __launch_bounds__(384, 1)
             } else {
 #pragma unroll
             for (int half = 0; half < D / 64; ++half) {
-                // the staging buffer is free once the bulk store that read it last is done
-                if (lane == 0) bulk_wait_read_all();
-                __syncwarp();
-                // this lane's row, columns [64*half, 64*half + 64): 128 bytes as 8
-                // chunks of 16; chunk i of row r sits at slot i ^ (r & 7), the layout
-                // of a 128-byte-swizzled 32-row box of O
+                // this lane's row, columns [64*half, 64*half + 64), read and rounded
+                // before waiting for the staging buffer, so the TMEM loads overlap
+                // the previous bulk store's read of it
+                uint4 v4[8];
 #pragma unroll
                 for (int c2 = 0; c2 < 2; ++c2) {
                     const int c = half * 2 + c2;
@@ -757,16 +755,21 @@ __global__ void __launch_bounds__(384, 1)
                         if (lane == 0) mbar_arrive(&o_free[t]);
                     }
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int chunk = c2 * 4 + i;
-                        const uint4 v4 = make_uint4(
+                    for (int i = 0; i < 4; ++i)
+                        v4[c2 * 4 + i] = make_uint4(
                             E::pack2(__uint_as_float(r3[8 * i + 0]) * inv_l, __uint_as_float(r3[8 * i + 1]) * inv_l),
                             E::pack2(__uint_as_float(r3[8 * i + 2]) * inv_l, __uint_as_float(r3[8 * i + 3]) * inv_l),
                             E::pack2(__uint_as_float(r3[8 * i + 4]) * inv_l, __uint_as_float(r3[8 * i + 5]) * inv_l),
                             E::pack2(__uint_as_float(r3[8 * i + 6]) * inv_l, __uint_as_float(r3[8 * i + 7]) * inv_l));
-                        *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = v4;
-                    }
                 }
+                // the staging buffer is free once the bulk store that read it last is done
+                if (lane == 0) bulk_wait_read_all();
+                __syncwarp();
+                // 128 bytes as 8 chunks of 16; chunk i of row r sits at slot i ^ (r & 7),
+                // the layout of a 128-byte-swizzled 32-row box of O
+#pragma unroll
+                for (int chunk = 0; chunk < 8; ++chunk)
+                    *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = v4[chunk];
                 // one bulk tensor store of the warp's 32 rows x 64 columns (rows past N
                 // are clipped by the tensor map); the warp goes on at once
                 fence_proxy_async_smem();
