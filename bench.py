@@ -74,10 +74,10 @@ NCU_TRAFFIC = {
     "decode": {"bytes_per_launch": 536959744 + 3461376, "source_sha": "eaaf414296e5590d"},
     "decode_b1_l32k": {"bytes_per_launch": 134302976 + 3129856, "source_sha": "eaaf414296e5590d"},
     "decode_b8_l32k": {"bytes_per_launch": 1073927168 + 3971072, "source_sha": "eaaf414296e5590d"},
-    "attn_fwd_causal": {"bytes_per_launch": 133972736 + 13311744, "source_sha": "4f828c62cb3836c8"},
+    "attn_fwd_causal": {"bytes_per_launch": 141966080 + 13459968, "source_sha": "0fb1c2cb5c296374"},
     # the non-causal call is two launches at this shape (the plain kernel, then the last round in
     # 128-row halves): their sum
-    "attn_fwd_noncausal": {"bytes_per_launch": 87889408 + 6636544 + 13960192 + 0, "source_sha": "4f828c62cb3836c8"},
+    "attn_fwd_noncausal": {"bytes_per_launch": 87900416 + 9707008 + 13959680 + 0, "source_sha": "0fb1c2cb5c296374"},
 }
 
 
