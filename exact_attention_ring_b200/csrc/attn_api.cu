@@ -107,6 +107,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 // The combine keeps one weight per split in dynamic shared memory; with its few
 // static words it must stay under the 48 KiB a launch gets without opting in.
 constexpr int kCombineMaxSplits = 12000;
+// Longest sequence (N or L) a call accepts: counts rounded up to 256-row blocks
+// or 128-key tiles (N + 255, L + S - 1, ...) then stay within int.
+constexpr int kMaxSeq = 0x7fffffff - 255;
 
 template <int D, bool CAUSAL, bool F32OUT, class E, bool SPLIT>
 attn_status_t launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -206,7 +209,8 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
                        int N, int d, int causal, float scale, attn_stream_t stream) {
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return ATTN_ERR_INVALID_ARG;
-    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || (causal != 0 && causal != 1) || !scale_ok(scale))
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || N > kMaxSeq || Hq % Hkv != 0 || (causal != 0 && causal != 1) ||
+        !scale_ok(scale))
         return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (static_cast<long long>(B) * Hq > 65535LL * 1024) return ATTN_ERR_INVALID_ARG;
@@ -268,8 +272,8 @@ attn_status_t decode_impl(const void* q, const void* k, const void* v, float* o_
                                   attn_stream_t stream) {
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part) || !aligned16(lse_part))
         return ATTN_ERR_INVALID_ARG;
-    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0 || num_splits < 1 || num_splits > L ||
-        !scale_ok(scale))
+    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || L > kMaxSeq || Hq % Hkv != 0 || num_splits < 1 ||
+        num_splits > L || !scale_ok(scale))
         return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (B > 65535 || num_splits > 0x7fffffff / 2) return ATTN_ERR_INVALID_ARG;
@@ -394,7 +398,8 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
     const void* ptrs[] = {q, k, v, o, lse, dout, delta, dq, dk, dv};
     for (const void* ptr : ptrs)
         if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
-    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || (causal != 0 && causal != 1) || !scale_ok(scale))
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || N > kMaxSeq || Hq % Hkv != 0 || (causal != 0 && causal != 1) ||
+        !scale_ok(scale))
         return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     // the tile kernels' grid is (planes, 128-row tiles): both within 65535
@@ -423,7 +428,8 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
 attn_status_t attn_quant_fp8(const void* x, void* codes, float* scales, int planes, int N, int d, int per_plane,
                              int transpose, attn_stream_t stream) {
     if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return ATTN_ERR_INVALID_ARG;
-    if (planes < 1 || N < 1 || (per_plane != 0 && per_plane != 1) || (transpose != 0 && transpose != 1))
+    if (planes < 1 || N < 1 || N > kMaxSeq || (per_plane != 0 && per_plane != 1) ||
+        (transpose != 0 && transpose != 1))
         return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     const int nblk = (N + 127) / 128;
@@ -457,7 +463,7 @@ attn_status_t attn_quant_fp8(const void* x, void* codes, float* scales, int plan
 attn_status_t attn_quant_fp8_rotate(const void* x, const float* signs, void* codes, float* scales, int planes, int N,
                                     int d, attn_stream_t stream) {
     if (!aligned16(x) || !aligned16(signs) || !aligned16(codes) || !aligned16(scales)) return ATTN_ERR_INVALID_ARG;
-    if (planes < 1 || N < 1 || planes > 65535) return ATTN_ERR_INVALID_ARG;
+    if (planes < 1 || N < 1 || N > kMaxSeq || planes > 65535) return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     const int nblk = (N + 127) / 128;
     QuantParams p{};
@@ -480,7 +486,8 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, cons
     const void* ptrs[] = {q8, k8, vt8, sq, sk, sv, o, lse};
     for (const void* ptr : ptrs)
         if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
-    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || (causal != 0 && causal != 1) || !scale_ok(scale))
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || N > kMaxSeq || Hq % Hkv != 0 || (causal != 0 && causal != 1) ||
+        !scale_ok(scale))
         return ATTN_ERR_INVALID_ARG;
     if (d != 128) return ATTN_ERR_UNSUPPORTED;
     if (static_cast<long long>(B) * Hq > 65535LL) return ATTN_ERR_INVALID_ARG;
@@ -517,7 +524,7 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, cons
 }
 
 int attn_decode_default_splits(int B, int Hq, int Hkv, int L) {
-    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0) return 0;
+    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || L > kMaxSeq || Hq % Hkv != 0) return 0;
     // Decode blocks (one per SM, 148 on B200; two per SM for the keys-as-rows
     // kernel with a 3-slot ring) each stream their split at about their share of
     // HBM bandwidth after a fixed start-up worth ~260 keys. Pick the split count
@@ -606,7 +613,8 @@ extern "C" attn_status_t attn_decode_noalloc(const void* q, const void* k, const
                                              attn_stream_t stream) {
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return ATTN_ERR_INVALID_ARG;
-    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || num_splits < 1 || num_splits > L) return ATTN_ERR_INVALID_ARG;
+    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || L > kMaxSeq || num_splits < 1 || num_splits > L)
+        return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     // every limit of the two launches is checked here, so that nothing is
     // enqueued unless both can run

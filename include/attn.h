@@ -25,6 +25,9 @@
  *  - Every pointer must be 16-byte aligned and must not alias another argument.
  *  - Arguments are checked before anything is launched; a failed check returns a
  *    status and enqueues nothing. A launch failure returns ATTN_ERR_CUDA.
+ *  - Sequence lengths (N, L) are at most 2^31 - 256, so that the block and tile
+ *    counts rounded up from them fit an int; a longer one is
+ *    ATTN_ERR_INVALID_ARG (attn_decode_default_splits returns 0).
  *  - Every wait inside a kernel is bounded. A kernel whose wait runs out records
  *    ATTN_ERR_TIMEOUT in a device-side status word and returns early (its outputs
  *    are then undefined); attn_device_status() reads and clears that word.

@@ -270,3 +270,37 @@ def test_fwd_fp8_rejects_invalid(lib, kw):
 @pytest.mark.parametrize("d", [64, 96, 256])
 def test_fwd_fp8_rejects_unsupported_head_dim(lib, d):
     assert _fwd8(lib, d=d) == UNSUPPORTED
+
+
+def _rot8(lib, x=16, signs=32, c=48, s=64, planes=2, N=100, d=128):
+    P = ctypes.c_void_p
+    lib.attn_quant_fp8_rotate.restype = ctypes.c_int
+    return lib.attn_quant_fp8_rotate(P(x), P(signs), P(c), P(s), planes, N, d, None)
+
+
+@pytest.mark.parametrize("kw", [dict(x=0), dict(signs=0), dict(signs=36), dict(c=0), dict(s=0), dict(planes=0),
+                                dict(N=0), dict(planes=70000)])
+def test_quant_fp8_rotate_rejects_invalid(lib, kw):
+    assert _rot8(lib, **kw) == INVALID
+
+
+# The longest sequence a call takes is 2^31 - 256: the 256-row block and 128-key
+# tile counts rounded up from it still fit an int. One row more is rejected
+# before anything is launched.
+TOO_LONG = 2**31 - 255
+
+
+def test_sequence_longer_than_the_limit_is_rejected(lib):
+    assert _fwd(lib, N=TOO_LONG) == INVALID
+    assert _fwd32(lib, N=TOO_LONG) == INVALID
+    assert _fwd16(lib, N=TOO_LONG) == INVALID
+    assert _bwd(lib, N=TOO_LONG) == INVALID
+    assert _dec(lib, L=TOO_LONG) == INVALID
+    assert _dec16(lib, L=TOO_LONG) == INVALID
+    assert _quant8(lib, N=TOO_LONG) == INVALID
+    assert _rot8(lib, N=TOO_LONG) == INVALID
+    assert _fwd8(lib, N=TOO_LONG) == INVALID
+    f = lib.attn_decode_default_splits
+    f.restype = ctypes.c_int
+    assert f(1, 32, 8, TOO_LONG) == 0
+    assert f(1, 32, 8, TOO_LONG - 1) > 0

@@ -94,3 +94,16 @@ def test_noalloc_rejects_more_splits_than_the_combine_takes(lib):
     assert eab.attn_device_status() == ATTN_OK
     o_or, lse_or = oracle.decode(q.cpu(), k.cpu(), v.cpu(), d ** -0.5)
     assert_attn_close(o, lse, o_or, lse_or, "noalloc 12000 splits")
+
+
+def test_noalloc_rejects_a_sequence_past_the_length_limit(lib):
+    # L = 2^31 - 255, one key past the longest sequence any call takes: rejected
+    # before anything is enqueued, so small buffers stand in for the key/value arrays
+    q, k, v = (t.cuda() for t in si.make_decode(9400, 1, 1, 1, 128, 64))
+    o = torch.empty(1, 1, 64, device="cuda", dtype=torch.bfloat16)
+    lse = torch.empty(1, 1, device="cuda", dtype=torch.float32)
+    P = ctypes.c_void_p
+    st = lib.attn_decode_noalloc(P(q.data_ptr()), P(k.data_ptr()), P(v.data_ptr()), P(o.data_ptr()),
+                                 P(lse.data_ptr()), 1, 1, 1, 2**31 - 255, 64, 4, ctypes.c_float(0.125),
+                                 P(torch.cuda.current_stream().cuda_stream))
+    assert st == ATTN_ERR_INVALID_ARG
